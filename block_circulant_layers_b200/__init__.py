@@ -1,0 +1,31 @@
+"""B200-native rdFFT: in-place real-domain FFT and the block-circulant layer.
+
+Thin Python binding over the C ABI of include/rdfft.h (librdfft.so, built in-tree by
+``python -m block_circulant_layers_b200.build``). Every function marshals its
+arguments and calls the library; all of the computation runs in the library's CUDA
+kernels. There is no fallback: without the compiled library, importing the binding
+raises, and the functions accept CUDA tensors only.
+
+Tensor functions (torch is used for device memory and the current stream):
+    rdfft_fwd(t, p)                       in place, packed spectrum of each row
+    rdfft_inv(t, p)                       in place, inverse
+    circ_fwd(x, c_hat, p, y=None)         y = W x
+    circ_bwd(g, x, c_hat, p, grad_x=..., grad_c=...)
+    circ_prepare(c)                       c_hat = packed rdfft_fwd of fp32 c
+Raw entry points on integer device pointers: ``lib`` (the ctypes handle).
+"""
+from __future__ import annotations
+
+_EXPORTS = ("RDFFT_BF16", "RDFFT_F32", "RdfftError", "circ_bwd", "circ_fwd", "circ_prepare",
+            "lib", "lib_path", "rdfft_fwd", "rdfft_inv")
+
+__all__ = list(_EXPORTS)
+
+
+def __getattr__(name):
+    # Loaded on first use so that `python -m block_circulant_layers_b200.build` can run
+    # before the library exists; any use of the API without it raises ImportError.
+    if name in _EXPORTS:
+        from . import _binding
+        return getattr(_binding, name)
+    raise AttributeError(name)

@@ -1,0 +1,143 @@
+"""ctypes binding of librdfft.so (argument marshalling only)."""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(_HERE, "librdfft.so")
+
+RDFFT_F32 = 0
+RDFFT_BF16 = 1
+
+if not os.path.exists(lib_path):
+    raise ImportError(
+        f"{lib_path} is missing: build it with `python -m block_circulant_layers_b200.build` "
+        "(the package has no non-CUDA fallback)")
+
+lib = ctypes.CDLL(lib_path)
+
+_i64, _int, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+lib.rdfft_fwd.argtypes = [_vp, _i64, _int, _int, _vp]
+lib.rdfft_inv.argtypes = [_vp, _i64, _int, _int, _vp]
+lib.circ_fwd.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
+lib.circ_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _vp]
+for _f in (lib.rdfft_fwd, lib.rdfft_inv, lib.circ_fwd, lib.circ_bwd):
+    _f.restype = _int
+lib.rdfft_strerror.argtypes = [_int]
+lib.rdfft_strerror.restype = ctypes.c_char_p
+lib.rdfft_version.argtypes = []
+lib.rdfft_version.restype = _int
+
+
+class RdfftError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {lib.rdfft_strerror(code).decode()} (code {code})")
+
+
+def _check(code: int, where: str) -> None:
+    if code != 0:
+        raise RdfftError(code, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return RDFFT_F32
+    if t.dtype == torch.bfloat16:
+        return RDFFT_BF16
+    raise TypeError(f"rdfft supports float32 and bfloat16 tensors, got {t.dtype}")
+
+
+def _cuda_dense(t: torch.Tensor, name: str) -> None:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _stream(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def rdfft_fwd(t: torch.Tensor, p: int) -> torch.Tensor:
+    """In-place packed rdFFT of every length-p row of `t` (numel a multiple of p)."""
+    _cuda_dense(t, "t")
+    if p <= 0 or t.numel() % p:
+        raise ValueError("numel must be a multiple of p")
+    with torch.cuda.device(t.device):
+        _check(lib.rdfft_fwd(t.data_ptr(), t.numel() // p, p, _dtype_code(t), _stream(t)), "rdfft_fwd")
+    return t
+
+
+def rdfft_inv(t: torch.Tensor, p: int) -> torch.Tensor:
+    """In-place inverse rdFFT (with 1/p) of every packed length-p row of `t`."""
+    _cuda_dense(t, "t")
+    if p <= 0 or t.numel() % p:
+        raise ValueError("numel must be a multiple of p")
+    with torch.cuda.device(t.device):
+        _check(lib.rdfft_inv(t.data_ptr(), t.numel() // p, p, _dtype_code(t), _stream(t)), "rdfft_inv")
+    return t
+
+
+def circ_prepare(c: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """c_hat for circ_fwd / circ_bwd: the packed rdFFT of fp32 c (q x q x p)."""
+    _cuda_dense(c, "c")
+    if c.dim() != 3 or c.shape[0] != c.shape[1]:
+        raise ValueError("c must have shape (q, q, p)")
+    p = c.shape[2]
+    if out is None:
+        out = c.detach().to(torch.float32).clone()
+    else:
+        out.copy_(c)
+    return rdfft_fwd(out, p)
+
+
+def _layer_dims(x: torch.Tensor, p: int):
+    D = x.shape[-1]
+    B = x.numel() // D if D else 0
+    return B, D
+
+
+def circ_fwd(x: torch.Tensor, c_hat: torch.Tensor, p: int, y: torch.Tensor | None = None) -> torch.Tensor:
+    """y = W x of the block-circulant layer, for x of shape (..., D)."""
+    _cuda_dense(x, "x")
+    _cuda_dense(c_hat, "c_hat")
+    if c_hat.dtype != torch.float32:
+        raise TypeError("c_hat must be float32")
+    if y is None:
+        y = torch.empty_like(x)
+    _cuda_dense(y, "y")
+    if y.dtype != x.dtype or y.shape != x.shape:
+        raise ValueError("y must match x in shape and dtype")
+    B, D = _layer_dims(x, p)
+    with torch.cuda.device(x.device):
+        _check(lib.circ_fwd(x.data_ptr(), c_hat.data_ptr(), y.data_ptr(), B, D, p, _dtype_code(x),
+                            _stream(x)), "circ_fwd")
+    return y
+
+
+def circ_bwd(g: torch.Tensor, x: torch.Tensor, c_hat: torch.Tensor, p: int,
+             grad_x: torch.Tensor | None = None, grad_c: torch.Tensor | None = None,
+             need_grad_x: bool = True, need_grad_c: bool = True):
+    """(grad_x, grad_c) of the block-circulant layer for upstream gradient g."""
+    _cuda_dense(g, "g")
+    _cuda_dense(x, "x")
+    _cuda_dense(c_hat, "c_hat")
+    if c_hat.dtype != torch.float32:
+        raise TypeError("c_hat must be float32")
+    if x.dtype != g.dtype or x.shape != g.shape:
+        raise ValueError("g must match x in shape and dtype")
+    B, D = _layer_dims(x, p)
+    if need_grad_x and grad_x is None:
+        grad_x = torch.empty_like(g)
+    if need_grad_c and grad_c is None:
+        grad_c = torch.empty(c_hat.shape, dtype=torch.float32, device=c_hat.device)
+    gx_ptr = grad_x.data_ptr() if (need_grad_x and grad_x is not None) else None
+    gc_ptr = grad_c.data_ptr() if (need_grad_c and grad_c is not None) else None
+    with torch.cuda.device(x.device):
+        _check(lib.circ_bwd(g.data_ptr(), x.data_ptr(), c_hat.data_ptr(), gx_ptr, gc_ptr, B, D, p,
+                            _dtype_code(x), _stream(x)), "circ_bwd")
+    return (grad_x if need_grad_x else None), (grad_c if need_grad_c else None)

@@ -1,0 +1,421 @@
+// Block-circulant linear layer kernels (sm_100a): forward, grad_x and grad_c.
+//
+// "Memory-Efficient Training with In-Place FFT Implementation", paper-notes page,
+// "Circulant matrix training adaptation": y = IFFT(FFT(c) (.) FFT(x)) per circulant
+// block; the product of conjugate-symmetric spectra stays conjugate symmetric, so
+// every spectrum lives in the packed layout and every transform is the in-place
+// rdFFT of packed_fft.cuh. With D = q p:
+//     forward : y_i      = IFFT( sum_j  C_ij (.) X_j )
+//     grad_x  : grad_x_j = IFFT( sum_i conj(C_ij) (.) G_i )
+//     grad_c  : grad_c_ij = IFFT( sum_b G_i^b (.) conj(X_j^b) )
+// where C = c_hat (packed, fp32), X = rdFFT(x), G = rdFFT(g) per block.
+//
+// Kernel shapes (ours):
+//  * k_circ_x (forward and grad_x): a CTA owns TT tokens and a group of QI output
+//    blocks. It rdFFTs the TT*q input rows straight from HBM into an fp32 shared
+//    tile, contracts them against c_hat (read through L2) with CUDA-core FMA into
+//    registers, writes the output spectra over the tile and rdIFFTs them straight
+//    back to HBM. HBM traffic: the input, c_hat, the output.
+//  * k_circ_gc (grad_c): a persistent CTA owns a group of QJ input blocks j and a
+//    slice of the tokens; it keeps its part of the packed cross-spectrum
+//    S_ij = sum_b G_i conj(X_j) in registers across all its token tiles and adds it
+//    into grad_c once (fp32 red.add). grad_c is zeroed first and rdIFFT'd in place
+//    after, so the output buffer is the only global storage used.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "packed_fft.cuh"
+
+namespace rdfft {
+
+// ------------------------------------------------------------- tile row passes
+// Forward rdFFT of tile rows [0, NR): row r reads its input from src(r) (nullptr
+// means a row of zeros), the spectrum stays in the tile.
+template <int P, int NT, typename T, int K, typename SrcFn>
+__device__ __forceinline__ void fft_rows_rest(float* tile, int NR, SrcFn src) {
+  if constexpr (K < Plan<P>::NPASS) {
+    constexpr int TPR = Plan<P>::TPR, RPR = NT / TPR;
+    __syncthreads();
+    const int v = threadIdx.x % TPR;
+    for (int r = threadIdx.x / TPR; r < NR; r += RPR)
+      orbit_pass<P, K, false, 0, 0>(tile, r, v, (T*)nullptr, false);
+    fft_rows_rest<P, NT, T, K + 1>(tile, NR, src);
+  }
+}
+
+template <int P, int NT, typename T, typename SrcFn>
+__device__ __forceinline__ void fft_rows(float* tile, int NR, SrcFn src) {
+  constexpr int TPR = Plan<P>::TPR, RPR = NT / TPR;
+  static_assert(NT % TPR == 0, "threads per CTA must cover whole rows");
+  const int v = threadIdx.x % TPR;
+  for (int r = threadIdx.x / TPR; r < NR; r += RPR) {
+    const T* g = src(r);
+    fwd_pass0<P, T>(tile, r, v, g, g != nullptr);
+  }
+  fft_rows_rest<P, NT, T, 1>(tile, NR, src);
+}
+
+// Inverse rdFFT of tile rows [0, NR) (the tile already synchronised); row r is
+// written to dst(r) (nullptr: dropped).
+template <int P, int NT, typename T, int K, typename DstFn>
+__device__ __forceinline__ void ifft_rows(float* tile, int NR, DstFn dst) {
+  constexpr int NP = Plan<P>::NPASS;
+  constexpr int TPR = Plan<P>::TPR, RPR = NT / TPR;
+  if constexpr (K < NP) {
+    if constexpr (K > 0) __syncthreads();
+    const int v = threadIdx.x % TPR;
+    for (int r = threadIdx.x / TPR; r < NR; r += RPR) {
+      if constexpr (K == NP - 1) {
+        T* g = dst(r);
+        inv_pass0<P, T>(tile, r, v, g, g != nullptr);
+      } else {
+        orbit_pass<P, NP - 1 - K, true, 0, 0>(tile, r, v, (T*)nullptr, false);
+      }
+    }
+    ifft_rows<P, NT, T, K + 1>(tile, NR, dst);
+  }
+}
+
+// Packed-bin view of a row: bin 0 is the real pair (slot 0, slot p/2); bin k > 0 is
+// the complex value (slot k, slot p - k).
+template <int P>
+__device__ __forceinline__ int bin_im_slot(int k) { return k == 0 ? P / 2 : P - k; }
+
+// --------------------------------------------------------------- forward, grad_x
+// BWDX = false: in = x, out = y; the CTA's QI output blocks are i, summed over j.
+// BWDX = true : in = g, out = grad_x; the CTA's QI output blocks are j, summed over i,
+//               against conj(c_hat).
+template <int P, typename T, int NT, int TT, int NS, bool BWDX>
+__global__ void __launch_bounds__(NT)
+k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict__ out,
+         int64_t B, int q, int QI) {
+  extern __shared__ float tile[];
+  const int D = q * P;
+  const int64_t tok0 = (int64_t)blockIdx.x * TT;
+  const int ntok = (int)((B - tok0) < TT ? (B - tok0) : TT);
+  const int o0 = blockIdx.y * QI;            // first output block of this CTA
+
+  // 1. rdFFT of the TT*q input rows (row r = t*q + b)
+  fft_rows<P, NT, T>(tile, TT * q, [&](int r) -> const T* {
+    const int t = r / q, b = r - t * q;
+    return t < ntok ? in + (tok0 + t) * (int64_t)D + (int64_t)b * P : nullptr;
+  });
+  __syncthreads();
+
+  // 2. contraction: thread slot s covers bin k and output block ol of all TT tokens
+  constexpr int HB = P / 2;
+  float acc_r[NS][TT], acc_i[NS][TT];
+#pragma unroll
+  for (int s = 0; s < NS; ++s)
+#pragma unroll
+    for (int t = 0; t < TT; ++t) acc_r[s][t] = acc_i[s][t] = 0.0f;
+
+  // c_hat of the summed block j + 1 is loaded (through L2) while block j is
+  // contracted, so the L2 latency overlaps the FMA work.
+  float cr_n[NS], ci_n[NS];
+  auto load_c = [&](int j, float (&cr)[NS], float (&ci)[NS]) {
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const int pi = threadIdx.x + NT * s;
+      const int ol = pi / HB, k = pi % HB;
+      if (ol < QI) {
+        const int ob = o0 + ol;
+        const float* crow = chat + (int64_t)(BWDX ? (j * q + ob) : (ob * q + j)) * P;
+        cr[s] = __ldg(crow + k);
+        ci[s] = __ldg(crow + bin_im_slot<P>(k));
+      } else {
+        cr[s] = ci[s] = 0.0f;
+      }
+    }
+  };
+  load_c(0, cr_n, ci_n);
+  for (int j = 0; j < q; ++j) {                 // j: summed block (input j for fwd, output i for grad_x)
+    float cr_c[NS], ci_c[NS];
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      cr_c[s] = cr_n[s];
+      ci_c[s] = ci_n[s];
+    }
+    if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
+#pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const int pi = threadIdx.x + NT * s;
+      const int ol = pi / HB, k = pi % HB;
+      if (ol < QI) {
+        const float cr = cr_c[s], ci = ci_c[s];
+        // packed product: bin 0 multiplies the real pair component-wise, other bins
+        // are complex products (conjugated c for grad_x)
+        const bool z = (k == 0);
+        const float a2 = z ? 0.0f : (BWDX ? ci : -ci);
+        const float a3 = z ? ci : cr;
+        const float a4 = z ? 0.0f : (BWDX ? -ci : ci);
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          const int row = t * q + j;
+          const float xr = tile[Swz<P>::at(row * P + k)];
+          const float xi = tile[Swz<P>::at(row * P + bin_im_slot<P>(k))];
+          acc_r[s][t] = fmaf(cr, xr, fmaf(a2, xi, acc_r[s][t]));
+          acc_i[s][t] = fmaf(a3, xi, fmaf(a4, xr, acc_i[s][t]));
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // 3. output spectra over the tile: row t*QI + ol
+#pragma unroll
+  for (int s = 0; s < NS; ++s) {
+    const int pi = threadIdx.x + NT * s;
+    const int ol = pi / HB, k = pi % HB;
+    if (ol < QI) {
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const int row = t * QI + ol;
+        tile[Swz<P>::at(row * P + k)] = acc_r[s][t];
+        tile[Swz<P>::at(row * P + bin_im_slot<P>(k))] = acc_i[s][t];
+      }
+    }
+  }
+  __syncthreads();
+
+  // 4. rdIFFT of the TT*QI output rows straight to HBM
+  ifft_rows<P, NT, T, 0>(tile, TT * QI, [&](int r) -> T* {
+    const int t = r / QI, ol = r - t * QI;
+    return t < ntok ? out + (tok0 + t) * (int64_t)D + (int64_t)(o0 + ol) * P : nullptr;
+  });
+}
+
+// ---------------------------------------------------------------------- grad_c
+// Thread group gamma = (k, ib, jb): bin k, output blocks i = ib*RI .. +RI, input
+// blocks jl = jb*RJ .. +RJ of the CTA's QJ-block group. The tile holds, per token
+// tile, G for rows t*q + i and X for rows TT*q + t*QJ + jl.
+template <int P, typename T, int NT, int TT, int NG, int RI, int RJ>
+__global__ void __launch_bounds__(NT, 1)
+k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ grad_c,
+          int64_t B, int q, int QJ, int64_t tok_per_cta) {
+  extern __shared__ float tile[];
+  constexpr int HB = P / 2;
+  const int D = q * P;
+  const int j0 = blockIdx.y * QJ;
+  const int64_t tbeg = (int64_t)blockIdx.x * tok_per_cta;
+  const int64_t tend = (tbeg + tok_per_cta < B) ? tbeg + tok_per_cta : B;
+  const int nib = q / RI, njb = QJ / RJ;
+  const int ngroups = HB * nib * njb;
+
+  float s_r[NG][RI][RJ], s_i[NG][RI][RJ];
+#pragma unroll
+  for (int n = 0; n < NG; ++n)
+#pragma unroll
+    for (int a = 0; a < RI; ++a)
+#pragma unroll
+      for (int b = 0; b < RJ; ++b) s_r[n][a][b] = s_i[n][a][b] = 0.0f;
+
+  const int xrow0 = TT * q;
+  for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
+    const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
+    if (tok0 != tbeg) __syncthreads();          // previous tile fully consumed
+    // rows [0, TT*q): G; rows [TT*q, TT*q + TT*QJ): X of the CTA's blocks
+    fft_rows<P, NT, T>(tile, TT * q + TT * QJ, [&](int r) -> const T* {
+      if (r < xrow0) {
+        const int t = r / q, b = r - t * q;
+        return t < ntok ? g + (tok0 + t) * (int64_t)D + (int64_t)b * P : nullptr;
+      }
+      const int rr = r - xrow0;
+      const int t = rr / QJ, jl = rr - t * QJ;
+      return t < ntok ? x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
+    });
+    __syncthreads();
+#pragma unroll
+    for (int n = 0; n < NG; ++n) {
+      const int gam = threadIdx.x + NT * n;
+      if (gam < ngroups) {
+        const int k = gam % HB;
+        const int rest = gam / HB;
+        const int ib = rest % nib, jb = rest / nib;
+        const bool z = (k == 0);
+        const int kim = bin_im_slot<P>(k);
+        for (int t = 0; t < ntok; ++t) {
+          float gr[RI], gi[RI];
+#pragma unroll
+          for (int a = 0; a < RI; ++a) {
+            const int row = t * q + ib * RI + a;
+            gr[a] = tile[Swz<P>::at(row * P + k)];
+            gi[a] = tile[Swz<P>::at(row * P + kim)];
+          }
+#pragma unroll
+          for (int b = 0; b < RJ; ++b) {
+            const int row = xrow0 + t * QJ + jb * RJ + b;
+            const float xr = tile[Swz<P>::at(row * P + k)];
+            const float xi = tile[Swz<P>::at(row * P + kim)];
+            // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)
+            const float xi_re = z ? 0.0f : xi;
+            const float x_im = z ? xi : xr;
+            const float xi_im = z ? 0.0f : -xi;
+#pragma unroll
+            for (int a = 0; a < RI; ++a) {
+              s_r[n][a][b] = fmaf(gr[a], xr, fmaf(gi[a], xi_re, s_r[n][a][b]));
+              s_i[n][a][b] = fmaf(gi[a], x_im, fmaf(gr[a], xi_im, s_i[n][a][b]));
+            }
+          }
+        }
+      }
+    }
+  }
+  // add this CTA's partial packed cross-spectrum into grad_c
+#pragma unroll
+  for (int n = 0; n < NG; ++n) {
+    const int gam = threadIdx.x + NT * n;
+    if (gam < ngroups) {
+      const int k = gam % HB;
+      const int rest = gam / HB;
+      const int ib = rest % nib, jb = rest / nib;
+      const int kim = bin_im_slot<P>(k);
+#pragma unroll
+      for (int a = 0; a < RI; ++a)
+#pragma unroll
+        for (int b = 0; b < RJ; ++b) {
+          float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
+          atomicAdd(dst + k, s_r[n][a][b]);
+          atomicAdd(dst + kim, s_i[n][a][b]);
+        }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ launchers
+static int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess && cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && n > 0)
+    return n;
+  return 148;
+}
+
+template <typename KernelT>
+static cudaError_t set_smem(KernelT kernel, size_t bytes) {
+  if (bytes <= 48 * 1024) return cudaSuccess;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+static int largest_divisor_leq(int q, int cap) {
+  for (int d = cap; d >= 1; --d)
+    if (q % d == 0) return d;
+  return 1;
+}
+
+// Forward / grad_x: NT threads, TT tokens per CTA, NS bins per thread, so a CTA
+// covers up to NS*NT/(P/2) output blocks.
+template <int P, typename T, int NT, int TT, int NS, bool BWDX>
+static cudaError_t launch_x_cfg(const void* in, const float* chat, void* out, int64_t B, int q,
+                                cudaStream_t s) {
+  constexpr int QI_MAX = NS * NT / (P / 2);
+  static_assert(QI_MAX >= 1, "slots must cover one block");
+  const int QI = largest_divisor_leq(q, QI_MAX);
+  const size_t smem = sizeof(float) * (size_t)TT * q * P;
+  auto kern = k_circ_x<P, T, NT, TT, NS, BWDX>;
+  cudaError_t e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t gx = (B + TT - 1) / TT;
+  if (gx > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  dim3 grid((unsigned)gx, (unsigned)(q / QI));
+  kern<<<grid, NT, smem, s>>>(static_cast<const T*>(in), chat, static_cast<T*>(out), B, q, QI);
+  return cudaGetLastError();
+}
+
+// Launch policy (at most 32 complex accumulators per thread, NS * TT <= 32):
+//  p <= 512 : 256 threads, up to 8 output blocks per CTA, 1/2/4 tokens per CTA by B;
+//  p >= 1024: 128 threads, one token per CTA (4 for the q = 1, p = 1024 layer).
+template <int P, typename T, bool BWDX>
+static cudaError_t launch_x_p(const void* in, const float* chat, void* out, int64_t B, int q,
+                              cudaStream_t s) {
+  if constexpr (P <= 512) {
+    constexpr int NT = 256;
+    constexpr int NS = (8 * (P / 2)) / NT > 0 ? (8 * (P / 2)) / NT : 1;
+    if (B >= 256 && NS * 4 <= 32) return launch_x_cfg<P, T, NT, 4, NS, BWDX>(in, chat, out, B, q, s);
+    if (B >= 32) return launch_x_cfg<P, T, NT, 2, NS, BWDX>(in, chat, out, B, q, s);
+    return launch_x_cfg<P, T, NT, 1, NS, BWDX>(in, chat, out, B, q, s);
+  } else {
+    constexpr int NT = 128;
+    constexpr int NS1 = (P / 2) / NT;                       // one output block per CTA
+    constexpr int NSM = NS1 * 4 <= 32 ? NS1 * 4 : 32;      // up to 4 (p=1024/2048) or 2 (p=4096)
+    if constexpr (P == 1024) {
+      if (q == 1 && B >= 64) return launch_x_cfg<P, T, NT, 4, NS1, BWDX>(in, chat, out, B, q, s);
+    }
+    return launch_x_cfg<P, T, NT, 1, NSM, BWDX>(in, chat, out, B, q, s);
+  }
+}
+
+template <int P, typename T, int NT, int TT, int NG, int RI, int RJ>
+static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B, int q, int QJ,
+                          cudaStream_t s) {
+  auto kern = k_circ_gc<P, T, NT, TT, NG, RI, RJ>;
+  const size_t smem = sizeof(float) * (size_t)TT * (q + QJ) * P;
+  cudaError_t e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  const int njgroups = q / QJ;
+  int slices = (num_sms() + njgroups - 1) / njgroups;
+  const int64_t tiles = (B + TT - 1) / TT;
+  if (slices > tiles) slices = (int)tiles;
+  const int64_t tiles_per = (tiles + slices - 1) / slices;
+  slices = (int)((tiles + tiles_per - 1) / tiles_per);
+  dim3 grid((unsigned)slices, (unsigned)njgroups);
+  kern<<<grid, NT, smem, s>>>(static_cast<const T*>(g), static_cast<const T*>(x), grad_c, B, q, QJ,
+                              tiles_per * TT);
+  return cudaGetLastError();
+}
+
+// grad_c launcher: a CTA of 512 threads keeps S for QJ input blocks in registers,
+// RI x RJ (output, input) blocks of one bin per thread-slot, NG slots per thread,
+// at most 32 complex accumulators per thread.
+template <int P, typename T>
+static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int64_t B, int q,
+                               cudaStream_t s) {
+  constexpr int NT = 512;
+  constexpr int TT = (P >= 2048) ? 1 : 2;
+  constexpr int HB = P / 2;
+  int QJ = largest_divisor_leq(q, 8);
+  while (QJ > 1 && (int64_t)HB * q * QJ > 32LL * NT) QJ = largest_divisor_leq(q, QJ - 1);
+  if ((int64_t)HB * q * QJ > 32LL * NT) return cudaErrorInvalidConfiguration;
+  const int64_t slots = (int64_t)HB * q * QJ;                // complex accumulators per CTA
+  if (q % 4 == 0 && QJ % 8 == 0 && slots <= 32LL * NT) return run_gc<P, T, NT, TT, 1, 4, 8>(g, x, grad_c, B, q, QJ, s);
+  if (q % 4 == 0 && QJ % 4 == 0) {
+    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 1, 4, 4>(g, x, grad_c, B, q, QJ, s);
+    return run_gc<P, T, NT, TT, 2, 4, 4>(g, x, grad_c, B, q, QJ, s);
+  }
+  if (q % 2 == 0 && QJ % 2 == 0) {
+    if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 1, 2, 2>(g, x, grad_c, B, q, QJ, s);
+    if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 2, 2, 2>(g, x, grad_c, B, q, QJ, s);
+    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 4, 2, 2>(g, x, grad_c, B, q, QJ, s);
+    return run_gc<P, T, NT, TT, 8, 2, 2>(g, x, grad_c, B, q, QJ, s);
+  }
+  if (slots <= 1LL * NT) return run_gc<P, T, NT, TT, 1, 1, 1>(g, x, grad_c, B, q, QJ, s);
+  if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 4, 1, 1>(g, x, grad_c, B, q, QJ, s);
+  if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 8, 1, 1>(g, x, grad_c, B, q, QJ, s);
+  if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 16, 1, 1>(g, x, grad_c, B, q, QJ, s);
+  return run_gc<P, T, NT, TT, 32, 1, 1>(g, x, grad_c, B, q, QJ, s);
+}
+
+// Per-p entry of the layer, instantiated once per translation unit (circ_p*.cu):
+// op 0 = forward (a = x, out = y); op 1 = grad_x (a = g, out = grad_x);
+// op 2 = grad_c accumulation (a = g, b = x, gc = grad_c, zeroed by the caller).
+template <int P>
+cudaError_t circ_layer_p(int op, const void* a, const void* b, const float* chat, void* out, float* gc,
+                         int64_t B, int q, int dtype, cudaStream_t s) {
+  if (dtype == 0) {
+    if (op == 0) return launch_x_p<P, float, false>(a, chat, out, B, q, s);
+    if (op == 1) return launch_x_p<P, float, true>(a, chat, out, B, q, s);
+    return launch_gc_p<P, float>(a, b, gc, B, q, s);
+  }
+  if (op == 0) return launch_x_p<P, bf16_t, false>(a, chat, out, B, q, s);
+  if (op == 1) return launch_x_p<P, bf16_t, true>(a, chat, out, B, q, s);
+  return launch_gc_p<P, bf16_t>(a, b, gc, B, q, s);
+}
+
+#define RDFFT_CIRC_INSTANCE(PP)                                                                  \
+  cudaError_t circ_layer_##PP(int op, const void* a, const void* b, const float* chat, void* out, \
+                              float* gc, int64_t B, int q, int dtype, cudaStream_t s) {           \
+    return circ_layer_p<PP>(op, a, b, chat, out, gc, B, q, dtype, s);                             \
+  }
+
+}  // namespace rdfft

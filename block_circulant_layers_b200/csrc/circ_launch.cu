@@ -1,0 +1,50 @@
+// Block-circulant layer: dispatch on the block size p and the backward sequence.
+#include <cuda_runtime.h>
+
+#include "internal.h"
+
+namespace rdfft {
+
+cudaError_t circ_layer_64(int, const void*, const void*, const float*, void*, float*, int64_t, int, int, cudaStream_t);
+cudaError_t circ_layer_128(int, const void*, const void*, const float*, void*, float*, int64_t, int, int, cudaStream_t);
+cudaError_t circ_layer_256(int, const void*, const void*, const float*, void*, float*, int64_t, int, int, cudaStream_t);
+cudaError_t circ_layer_512(int, const void*, const void*, const float*, void*, float*, int64_t, int, int, cudaStream_t);
+cudaError_t circ_layer_1024(int, const void*, const void*, const float*, void*, float*, int64_t, int, int, cudaStream_t);
+cudaError_t circ_layer_2048(int, const void*, const void*, const float*, void*, float*, int64_t, int, int, cudaStream_t);
+cudaError_t circ_layer_4096(int, const void*, const void*, const float*, void*, float*, int64_t, int, int, cudaStream_t);
+
+static cudaError_t circ_layer(int p, int op, const void* a, const void* b, const float* chat, void* out,
+                              float* gc, int64_t B, int q, int dtype, cudaStream_t s) {
+  switch (p) {
+    case 64: return circ_layer_64(op, a, b, chat, out, gc, B, q, dtype, s);
+    case 128: return circ_layer_128(op, a, b, chat, out, gc, B, q, dtype, s);
+    case 256: return circ_layer_256(op, a, b, chat, out, gc, B, q, dtype, s);
+    case 512: return circ_layer_512(op, a, b, chat, out, gc, B, q, dtype, s);
+    case 1024: return circ_layer_1024(op, a, b, chat, out, gc, B, q, dtype, s);
+    case 2048: return circ_layer_2048(op, a, b, chat, out, gc, B, q, dtype, s);
+    case 4096: return circ_layer_4096(op, a, b, chat, out, gc, B, q, dtype, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p,
+                            int dtype, cudaStream_t s) {
+  return circ_layer(p, 0, x, nullptr, c_hat, y, nullptr, B, D / p, dtype, s);
+}
+
+cudaError_t launch_circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x,
+                            float* grad_c, int64_t B, int D, int p, int dtype, cudaStream_t s) {
+  const int q = D / p;
+  cudaError_t e = cudaSuccess;
+  if (grad_c != nullptr) {
+    // zero, accumulate the packed cross-spectrum over all tokens, rdIFFT in place
+    e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)q * q * p, s);
+    if (e == cudaSuccess) e = circ_layer(p, 2, g, x, c_hat, nullptr, grad_c, B, q, dtype, s);
+    if (e == cudaSuccess) e = launch_rows(grad_c, (int64_t)q * q, p, 0, true, s);
+    if (e != cudaSuccess) return e;
+  }
+  if (grad_x != nullptr) e = circ_layer(p, 1, g, nullptr, c_hat, grad_x, nullptr, B, q, dtype, s);
+  return e;
+}
+
+}  // namespace rdfft

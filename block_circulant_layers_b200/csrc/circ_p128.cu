@@ -1,0 +1,6 @@
+// Block-circulant layer kernels for block size p = 128 (one translation unit per p).
+#include "circ_kernels.cuh"
+
+namespace rdfft {
+RDFFT_CIRC_INSTANCE(128)
+}  // namespace rdfft

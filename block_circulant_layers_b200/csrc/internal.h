@@ -1,0 +1,21 @@
+// Launchers shared between the C ABI layer and the kernel translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace rdfft {
+
+// Batched in-place rdFFT (inverse = false) or rdIFFT (inverse = true) of `rows`
+// rows of length p; dtype 0 = fp32, 1 = bf16. Arguments are already validated.
+cudaError_t launch_rows(void* data, int64_t rows, int p, int dtype, bool inverse, cudaStream_t s);
+
+// Block-circulant layer forward: y = W x (see circ_fwd in rdfft.h).
+cudaError_t launch_circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p,
+                            int dtype, cudaStream_t s);
+
+// Block-circulant layer backward (see circ_bwd in rdfft.h). grad_x / grad_c may be null.
+cudaError_t launch_circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x,
+                            float* grad_c, int64_t B, int D, int p, int dtype, cudaStream_t s);
+
+}  // namespace rdfft

@@ -1,0 +1,116 @@
+// C ABI of the library: argument validation and dispatch (declared in rdfft.h).
+// Every argument check happens before any CUDA call, so invalid calls enqueue
+// nothing and need no GPU.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "rdfft.h"
+#include "internal.h"
+
+namespace {
+
+thread_local cudaError_t t_last_cuda = cudaSuccess;
+thread_local char t_msg[256];
+
+bool pow2_in_range(int p) { return p >= 2 && p <= 4096 && (p & (p - 1)) == 0; }
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) == 0; }
+bool dtype_ok(int dtype) { return dtype == RDFFT_F32 || dtype == RDFFT_BF16; }
+
+int finish(cudaError_t e) {
+  if (e == cudaSuccess) return RDFFT_OK;
+  t_last_cuda = e;
+  return RDFFT_ECUDA;
+}
+
+int rows_call(void* data, int64_t rows, int p, int dtype, rdfft_stream_t stream, bool inverse) {
+  if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
+  if (!pow2_in_range(p) || rows < 0) return RDFFT_EINVAL;
+  if (rows == 0) return RDFFT_OK;
+  if (data == nullptr) return RDFFT_ENULL;
+  if (!aligned16(data)) return RDFFT_EALIGN;
+  return finish(rdfft::launch_rows(data, rows, p, dtype, inverse, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int layer_shape_ok(int64_t B, int D, int p) {
+  if (!pow2_in_range(p) || p < 64 || B < 0 || D < p || D > RDFFT_MAX_D || D % p != 0) return 0;
+  return 1;
+}
+
+// Byte ranges [a, a + na) and [b, b + nb) intersect (null pointers never do).
+bool overlap(const void* a, size_t na, const void* b, size_t nb) {
+  if (a == nullptr || b == nullptr || na == 0 || nb == 0) return false;
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rdfft_fwd(void* data, int64_t rows, int p, int dtype, rdfft_stream_t stream) {
+  return rows_call(data, rows, p, dtype, stream, false);
+}
+
+int rdfft_inv(void* data, int64_t rows, int p, int dtype, rdfft_stream_t stream) {
+  return rows_call(data, rows, p, dtype, stream, true);
+}
+
+int circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p, int dtype,
+             rdfft_stream_t stream) {
+  if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
+  if (!layer_shape_ok(B, D, p)) return RDFFT_EINVAL;
+  if (B == 0) return RDFFT_OK;
+  if (x == nullptr || c_hat == nullptr || y == nullptr) return RDFFT_ENULL;
+  if (!aligned16(x) || !aligned16(c_hat) || !aligned16(y)) return RDFFT_EALIGN;
+  const size_t act = (size_t)B * D * (dtype == RDFFT_F32 ? 4 : 2);
+  const size_t cb = sizeof(float) * (size_t)(D / p) * (D / p) * p;
+  if (overlap(y, act, x, act) || overlap(y, act, c_hat, cb)) return RDFFT_EOVERLAP;
+  return finish(rdfft::launch_circ_fwd(x, c_hat, y, B, D, p, dtype, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
+             int64_t B, int D, int p, int dtype, rdfft_stream_t stream) {
+  if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
+  if (!layer_shape_ok(B, D, p)) return RDFFT_EINVAL;
+  if (grad_x == nullptr && grad_c == nullptr) return RDFFT_OK;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t cb = sizeof(float) * (size_t)(D / p) * (D / p) * p;
+  if (B == 0) {
+    // no tokens: grad_x is empty and grad_c is an empty sum
+    if (grad_c == nullptr) return RDFFT_OK;
+    if (!aligned16(grad_c)) return RDFFT_EALIGN;
+    return finish(cudaMemsetAsync(grad_c, 0, cb, s));
+  }
+  if (g == nullptr || c_hat == nullptr) return RDFFT_ENULL;
+  if (grad_c != nullptr && x == nullptr) return RDFFT_ENULL;
+  if (!aligned16(g) || !aligned16(c_hat) || (x && !aligned16(x)) || (grad_x && !aligned16(grad_x)) ||
+      (grad_c && !aligned16(grad_c)))
+    return RDFFT_EALIGN;
+  const size_t act = (size_t)B * D * (dtype == RDFFT_F32 ? 4 : 2);
+  if (overlap(grad_x, act, g, act) || overlap(grad_x, act, x, act) || overlap(grad_x, act, c_hat, cb) ||
+      overlap(grad_x, act, grad_c, cb) || overlap(grad_c, cb, g, act) || overlap(grad_c, cb, x, act) ||
+      overlap(grad_c, cb, c_hat, cb))
+    return RDFFT_EOVERLAP;
+  return finish(rdfft::launch_circ_bwd(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, s));
+}
+
+const char* rdfft_strerror(int code) {
+  switch (code) {
+    case RDFFT_OK: return "ok";
+    case RDFFT_EINVAL: return "invalid size: p must be a power of two in [2, 4096] (>= 64 for the layer), counts >= 0, D a multiple of p and <= RDFFT_MAX_D";
+    case RDFFT_ENULL: return "a required pointer is NULL";
+    case RDFFT_EALIGN: return "a pointer is not 16-byte aligned";
+    case RDFFT_EDTYPE: return "dtype must be RDFFT_F32 (0) or RDFFT_BF16 (1)";
+    case RDFFT_EOVERLAP: return "an output buffer overlaps an input buffer";
+    case RDFFT_ECUDA:
+      snprintf(t_msg, sizeof(t_msg), "CUDA error while enqueuing: %s (%d)", cudaGetErrorString(t_last_cuda),
+               (int)t_last_cuda);
+      return t_msg;
+    default: return "unknown rdfft error code";
+  }
+}
+
+int rdfft_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,78 @@
+// Standalone batched rdFFT / rdIFFT kernels (sm_100a) and their launcher.
+//
+// One CTA of 128 threads owns a run of consecutive rows: for p >= 64 it owns
+// 128 / (p/32) rows with p/32 threads per row and an fp32 shared tile of 16 KiB;
+// for p <= 32 one thread owns one row. Every element is read once from HBM and
+// written once, in place; no other global memory is touched apart from the twiddle
+// tables, which stay in L1 / the constant cache.
+#include <cuda_runtime.h>
+
+#include "internal.h"
+#include "rdfft_steps.cuh"
+
+namespace rdfft {
+
+template <int P, bool INV, int K, typename T>
+__device__ __forceinline__ void run_steps(float* tile, int lrow, int v, T* g, bool active) {
+  if constexpr (K < Plan<P>::NPASS) {
+    if constexpr (K > 0) __syncthreads();
+    row_step<P, INV, K, T>(tile, lrow, v, g, active);
+    run_steps<P, INV, K + 1, T>(tile, lrow, v, g, active);
+  }
+}
+
+template <int P, bool INV, typename T>
+__global__ void __launch_bounds__(RowTiling<P>::THREADS)
+k_rows(T* __restrict__ data, int64_t rows) {
+  constexpr int ROWS = RowTiling<P>::ROWS;
+  if constexpr (P <= 32) {
+    const int64_t row = (int64_t)blockIdx.x * ROWS + threadIdx.x;
+    if (row < rows) row_small<P, INV, T>(data + row * P);
+  } else {
+    constexpr int TPR = Plan<P>::TPR;
+    __shared__ float tile[ROWS * P];
+    const int lrow = threadIdx.x / TPR;
+    const int v = threadIdx.x % TPR;
+    const int64_t row = (int64_t)blockIdx.x * ROWS + lrow;
+    const bool active = row < rows;
+    T* g = data + (active ? row : (int64_t)0) * P;
+    run_steps<P, INV, 0, T>(tile, lrow, v, g, active);
+  }
+}
+
+template <int P, typename T>
+static cudaError_t launch_p(void* data, int64_t rows, bool inverse, cudaStream_t s) {
+  constexpr int ROWS = RowTiling<P>::ROWS;
+  const int64_t grid = (rows + ROWS - 1) / ROWS;
+  if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  T* d = static_cast<T*>(data);
+  if (inverse) k_rows<P, true, T><<<(unsigned)grid, RowTiling<P>::THREADS, 0, s>>>(d, rows);
+  else k_rows<P, false, T><<<(unsigned)grid, RowTiling<P>::THREADS, 0, s>>>(d, rows);
+  return cudaGetLastError();
+}
+
+template <typename T>
+static cudaError_t launch_t(void* data, int64_t rows, int p, bool inverse, cudaStream_t s) {
+  switch (p) {
+    case 2: return launch_p<2, T>(data, rows, inverse, s);
+    case 4: return launch_p<4, T>(data, rows, inverse, s);
+    case 8: return launch_p<8, T>(data, rows, inverse, s);
+    case 16: return launch_p<16, T>(data, rows, inverse, s);
+    case 32: return launch_p<32, T>(data, rows, inverse, s);
+    case 64: return launch_p<64, T>(data, rows, inverse, s);
+    case 128: return launch_p<128, T>(data, rows, inverse, s);
+    case 256: return launch_p<256, T>(data, rows, inverse, s);
+    case 512: return launch_p<512, T>(data, rows, inverse, s);
+    case 1024: return launch_p<1024, T>(data, rows, inverse, s);
+    case 2048: return launch_p<2048, T>(data, rows, inverse, s);
+    case 4096: return launch_p<4096, T>(data, rows, inverse, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_rows(void* data, int64_t rows, int p, int dtype, bool inverse, cudaStream_t s) {
+  if (dtype == 0) return launch_t<float>(data, rows, p, inverse, s);
+  return launch_t<bf16_t>(data, rows, p, inverse, s);
+}
+
+}  // namespace rdfft

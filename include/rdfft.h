@@ -1,0 +1,142 @@
+/*
+ * rdfft.h -- C ABI of the B200 (sm_100a) rdFFT library: a real-domain, fully
+ * in-place FFT / IFFT over batched rows, and the block-circulant linear layer it
+ * drives, forward and backward.
+ *
+ * Source of the method: "Memory-Efficient Training with In-Place FFT
+ * Implementation" (arXiv 2511.01385). Citations below name the web page that
+ * describes a step and its section:
+ *   [summary]     the AI-written summary page, sections "Approach" and "Problem";
+ *   [notes]       the paper-notes page, method section, items "Squeeze N+2 -> N",
+ *                 "Proposition 1", "In-place IFFT design" and "Circulant matrix
+ *                 training adaptation", and its "Training strategy" list.
+ *
+ * Packed layout of a row of length p (every transform buffer uses it)
+ * ([summary] Approach; [notes] "Squeeze N+2 -> N"): the spectrum Y of a real row
+ * is conjugate symmetric, so it is stored in the row's own p slots:
+ *     slot 0     = Y_0            (real)
+ *     slot p/2   = Y_{p/2}        (real)
+ *     slot k     = Re Y_k         for 0 < k < p/2
+ *     slot p - k = Im Y_k         for 0 < k < p/2
+ * with Y_k = sum_n x_n exp(-2 pi i k n / p). For p = 2 the row is [Y_0, Y_1].
+ *
+ * Conventions shared by every entry point:
+ *   - All data pointers are DEVICE pointers owned by the caller, 16-byte aligned,
+ *     to dense row-major arrays. The library allocates no memory of any kind; its
+ *     only state is a read-only twiddle table built into the module image.
+ *   - `dtype` is RDFFT_F32 (float) or RDFFT_BF16 (bfloat16 raw bits, uint16). The
+ *     arithmetic is fp32 in both cases; bf16 results are rounded once, to nearest
+ *     even, when they are stored.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream) of the current
+ *     device. Calls are asynchronous on it: they validate their arguments, enqueue
+ *     kernels and return. They keep no state between calls and may be made from
+ *     several host threads at once.
+ *   - Return value: RDFFT_OK, or an error code. Argument errors are reported before
+ *     anything is enqueued. RDFFT_ECUDA means a CUDA call failed when enqueuing;
+ *     rdfft_strerror() then includes the CUDA message, which is kept per host
+ *     thread. Empty work (rows == 0 or B == 0) returns RDFFT_OK and enqueues nothing.
+ */
+#ifndef RDFFT_H
+#define RDFFT_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t, declared without the CUDA headers. */
+typedef struct CUstream_st* rdfft_stream_t;
+
+enum {
+  RDFFT_F32 = 0,
+  RDFFT_BF16 = 1
+};
+
+enum {
+  RDFFT_OK = 0,
+  RDFFT_EINVAL = 1,   /* p not a power of two in [2, 4096] ([64, 4096] for the layer); negative count; D % p != 0; D too large */
+  RDFFT_ENULL = 2,    /* a required pointer is NULL */
+  RDFFT_EALIGN = 3,   /* a pointer is not 16-byte aligned */
+  RDFFT_EDTYPE = 4,   /* dtype is neither RDFFT_F32 nor RDFFT_BF16 */
+  RDFFT_ECUDA = 5,    /* a CUDA call failed while enqueuing work */
+  RDFFT_EOVERLAP = 6  /* an output buffer overlaps an input buffer it may not alias */
+};
+
+/* Largest feature size D accepted by circ_fwd / circ_bwd. */
+#define RDFFT_MAX_D 8192
+
+/*
+ * rdfft_fwd -- forward rdFFT of `rows` rows of length p, in place.
+ * [notes] "Squeeze N+2 -> N" and "Proposition 1": radix-2 Cooley-Tukey whose
+ * butterflies act on four-element groups symmetric about a centre index, so the
+ * spectrum of each row overwrites the row in the packed layout above.
+ *   data  : rows x p elements of `dtype`; read as real rows, overwritten by their
+ *           packed spectra (unnormalised).
+ *   rows  : number of rows (>= 0).   p : row length, power of two in [2, 4096].
+ */
+int rdfft_fwd(void* data, int64_t rows, int p, int dtype, rdfft_stream_t stream);
+
+/*
+ * rdfft_inv -- inverse rdFFT (rdIFFT) of `rows` packed rows of length p, in place.
+ * [notes] "In-place IFFT design": the forward graph run backwards, each conjugate
+ * pair split into its symmetric and antisymmetric parts, x_a = (y_a + y_b)/2,
+ * x_b = (y_a - y_b)/(2 W). The product of those halvings is the 1/p of the inverse
+ * DFT, so rdfft_inv(rdfft_fwd(x)) = x up to rounding.
+ *   data  : rows x p packed spectra of `dtype`, overwritten by the real rows.
+ */
+int rdfft_inv(void* data, int64_t rows, int p, int dtype, rdfft_stream_t stream);
+
+/*
+ * circ_fwd -- block-circulant linear layer, forward.
+ * [notes] "Circulant matrix training adaptation": y = IFFT(FFT(c) (.) FFT(x)); the
+ * product of two conjugate-symmetric spectra is conjugate symmetric, so the packed
+ * layout carries it. With D = q p, block j of a token is x_j = x[j p, (j+1) p) and
+ *     y_i = IFFT( sum_{j<q} FFT(c_ij) (.) FFT(x_j) ),   i < q,
+ * i.e. y = W x where block (i, j) of W is the p x p circulant whose first column is
+ * c_ij.
+ *   x     : B x D of `dtype`, read only.
+ *   c_hat : q x q x p fp32, the packed rdfft_fwd of the fp32 parameters c[i][j][:]
+ *           (the caller runs rdfft_fwd on an fp32 copy of c; i = output block,
+ *           j = input block). Read only.
+ *   y     : B x D of `dtype`, written. y must not overlap x or c_hat
+ *           (RDFFT_EOVERLAP): several CTAs read each token row of x while others
+ *           already write output blocks of the same row.
+ *   B     : tokens (>= 0).  D : features, a multiple of p, D <= RDFFT_MAX_D.
+ *   p     : block size, power of two in [64, 4096] for the layer.
+ */
+int circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p, int dtype,
+             rdfft_stream_t stream);
+
+/*
+ * circ_bwd -- block-circulant linear layer, backward, for upstream gradient g = dL/dy.
+ * [notes] "Circulant matrix training adaptation" (gradients keep the symmetry) and
+ * "Training strategy" (forward and backward both in the real domain):
+ *     grad_x_j = IFFT( sum_i conj(FFT(c_ij)) (.) FFT(g_i) )            (= W^T g)
+ *     grad_c_ij = IFFT( sum_b FFT(g_i^b) (.) conj(FFT(x_j^b)) )        (summed over B)
+ *   g, x   : B x D of `dtype`, read only.
+ *   c_hat  : as in circ_fwd.
+ *   grad_x : B x D of `dtype`, written; may be NULL to skip it. Must not overlap
+ *            g, x, c_hat or grad_c (RDFFT_EOVERLAP).
+ *   grad_c : q x q x p fp32 in the spatial domain (same layout as c), overwritten
+ *            with the gradient summed over all B tokens; may be NULL to skip it.
+ *            The buffer is used in place: it is zeroed, accumulates the packed
+ *            cross-spectrum, and ends with an in-place rdIFFT of its q*q rows.
+ *            Must not overlap g, x or c_hat (RDFFT_EOVERLAP).
+ * The grad_c sum over tokens is accumulated with fp32 atomic adds, so its last bits
+ * may differ between runs; grad_x and the forward are deterministic.
+ */
+int circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
+             int64_t B, int D, int p, int dtype, rdfft_stream_t stream);
+
+/* Human-readable message for a return code (per host thread for RDFFT_ECUDA). */
+const char* rdfft_strerror(int code);
+
+/* Library version as 10000*major + 100*minor + patch. */
+int rdfft_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RDFFT_H */

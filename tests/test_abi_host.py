@@ -1,0 +1,111 @@
+"""C ABI checks that need no GPU: the library loads, exports every declared symbol,
+rejects bad arguments before touching CUDA, and its objects call no allocator."""
+import ctypes
+import glob
+import os
+import re
+import subprocess
+
+import pytest
+
+from conftest import ROOT
+
+PKG = os.path.join(ROOT, "block_circulant_layers_b200")
+HEADER = os.path.join(ROOT, "include", "rdfft.h")
+
+OK, EINVAL, ENULL, EALIGN, EDTYPE, ECUDA, EOVERLAP = range(7)
+F32, BF16 = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_circulant_layers_b200 import build
+    build.build_lib()
+    L = ctypes.CDLL(os.path.join(PKG, "librdfft.so"))
+    i64, i, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
+    L.rdfft_fwd.argtypes = [vp, i64, i, i, vp]
+    L.rdfft_inv.argtypes = [vp, i64, i, i, vp]
+    L.circ_fwd.argtypes = [vp, vp, vp, i64, i, i, i, vp]
+    L.circ_bwd.argtypes = [vp, vp, vp, vp, vp, i64, i, i, i, vp]
+    L.rdfft_strerror.argtypes = [i]
+    L.rdfft_strerror.restype = ctypes.c_char_p
+    return L
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return re.findall(r"^\s*(?:int|const char\*)\s+(\w+)\s*\(", src, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for n in ("rdfft_fwd", "rdfft_inv", "circ_fwd", "circ_bwd", "rdfft_strerror", "rdfft_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", os.path.join(PKG, "librdfft.so")],
+                         capture_output=True, text=True, check=True).stdout
+    exported = {ln.split()[-1] for ln in out.splitlines() if ln.strip()}
+    for name in declared_functions():
+        assert name in exported, name
+
+
+def test_version_and_messages(lib):
+    assert lib.rdfft_version() >= 100
+    for code in range(7):
+        assert lib.rdfft_strerror(code)
+    assert b"unknown" in lib.rdfft_strerror(99)
+
+
+A = 0x10000          # aligned fake device addresses: validation fails before any use
+Bp = 0x20000000
+
+
+def test_rdfft_argument_errors(lib):
+    for fn in (lib.rdfft_fwd, lib.rdfft_inv):
+        assert fn(None, 0, 512, F32, None) == OK          # empty work: nothing enqueued
+        assert fn(None, 4, 512, F32, None) == ENULL
+        assert fn(A, 4, 3, F32, None) == EINVAL
+        assert fn(A, 4, 1, F32, None) == EINVAL
+        assert fn(A, 4, 8192, F32, None) == EINVAL
+        assert fn(A, -1, 512, F32, None) == EINVAL
+        assert fn(A, 4, 512, 2, None) == EDTYPE
+        assert fn(A + 4, 4, 512, BF16, None) == EALIGN
+
+
+def test_circ_argument_errors(lib):
+    D, p = 4096, 128
+    assert lib.circ_fwd(A, Bp, A + (1 << 26), 0, D, p, BF16, None) == OK
+    assert lib.circ_fwd(A, Bp, A + (1 << 26), 4, 4000, p, BF16, None) == EINVAL   # D % p
+    assert lib.circ_fwd(A, Bp, A + (1 << 26), 4, 16384, p, BF16, None) == EINVAL  # D too large
+    assert lib.circ_fwd(A, Bp, A + (1 << 26), 4, 1024, 32, BF16, None) == EINVAL  # p < 64
+    assert lib.circ_fwd(A, Bp, A + (1 << 26), 4, D, p, 5, None) == EDTYPE
+    assert lib.circ_fwd(None, Bp, A, 4, D, p, BF16, None) == ENULL
+    assert lib.circ_fwd(A, None, A + (1 << 26), 4, D, p, BF16, None) == ENULL
+    assert lib.circ_fwd(A, Bp + 8, A + (1 << 26), 4, D, p, BF16, None) == EALIGN
+    assert lib.circ_fwd(A, Bp, A, 4, D, p, BF16, None) == EOVERLAP                 # y == x
+    assert lib.circ_fwd(A, Bp, A + 4096, 4, D, p, BF16, None) == EOVERLAP          # partial overlap
+    # backward
+    assert lib.circ_bwd(A, A, Bp, None, None, 4, D, p, BF16, None) == OK           # nothing asked
+    assert lib.circ_bwd(None, A, Bp, A + (1 << 26), None, 4, D, p, BF16, None) == ENULL
+    assert lib.circ_bwd(A, None, Bp, None, Bp + (1 << 24), 4, D, p, BF16, None) == ENULL
+    assert lib.circ_bwd(A, A, Bp, A, None, 4, D, p, BF16, None) == EOVERLAP        # grad_x == g
+    assert lib.circ_bwd(A, A + (1 << 25), Bp, None, A, 4, D, p, BF16, None) == EOVERLAP
+    assert lib.circ_bwd(A, A + (1 << 25), Bp, A + (1 << 26), None, 4, 4000, p, BF16, None) == EINVAL
+
+
+def test_objects_call_no_allocator():
+    """The library allocates nothing: none of its own objects references an allocator."""
+    from block_circulant_layers_b200 import build
+    build.build_lib()
+    objs = glob.glob(os.path.join(PKG, "_build", "*.o"))
+    assert objs
+    for o in objs:
+        und = subprocess.run(["nm", "-u", o], capture_output=True, text=True, check=True).stdout
+        for sym in ("cudaMalloc", "cudaMallocAsync", "cudaMallocManaged", "cudaMallocHost", "cuMemAlloc",
+                    "cudaHostAlloc", "cudaMallocPitch", "cudaMalloc3D"):
+            assert not re.search(rf"\b{sym}\w*\b", und), (o, sym)

@@ -1,0 +1,137 @@
+"""GPU parity of circ_fwd / circ_bwd (block-circulant layer) against the dense
+float64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import assert_parity, to_device, to_host_f64
+from synthetic import sample
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rd():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA GPU is required for the gpu tests")
+    import block_circulant_layers_b200 as rd
+    return rd
+
+
+def make_layer(B, D, p, dtype, seeds):
+    q = D // p
+    cs, xs, gs = seeds
+    c = sample(cs, (q, q, p), "f32", sigma=1.0 / np.sqrt(D))
+    x = sample(xs, (B, D), dtype)
+    g = sample(gs, (B, D), dtype)
+    return c, x, g
+
+
+def run_layer(rd, B, D, p, dtype, seeds, grads=True):
+    c, x, g = make_layer(B, D, p, dtype, seeds)
+    c_hat = rd.circ_prepare(to_device(c, "f32"))
+    xd, gd = to_device(x, dtype), to_device(g, dtype)
+    y = rd.circ_fwd(xd, c_hat, p)
+    gx = gc = None
+    if grads:
+        gx, gc = rd.circ_bwd(gd, xd, c_hat, p)
+    torch.cuda.synchronize()
+    return c, x, g, y, gx, gc
+
+
+def check_all(rd, B, D, p, dtype, seeds, tokens=None):
+    c, x, g, y, gx, gc = run_layer(rd, B, D, p, dtype, seeds)
+    sel = slice(None) if tokens is None else tokens
+    y_ref = oracle.circ_forward(x.exact[sel], c.exact)
+    assert_parity(to_host_f64(y)[sel], y_ref, dtype, f"y B={B} D={D} p={p}")
+    gx_ref, _ = oracle.circ_backward(g.exact[sel], x.exact[sel], c.exact)
+    assert_parity(to_host_f64(gx)[sel], gx_ref, dtype, f"grad_x B={B} D={D} p={p}")
+    _, gc_ref = oracle.circ_backward(g.exact, x.exact, c.exact)
+    assert_parity(to_host_f64(gc), gc_ref, dtype, f"grad_c B={B} D={D} p={p}")
+
+
+# small layers over every supported block size: several CTAs, ragged token counts
+SMALL = [(5, 256, 64), (7, 512, 128), (3, 1024, 256), (9, 1024, 512), (4, 2048, 1024),
+         (6, 4096, 2048), (5, 4096, 4096), (33, 512, 64), (70, 256, 128), (300, 128, 64)]
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("B,D,p", SMALL)
+def test_small_layers(rd, B, D, p, dtype):
+    check_all(rd, B, D, p, dtype, (100 + p, 200 + B, 300 + D))
+
+
+@pytest.mark.parametrize("D,p", [(768, 256), (3072, 1024), (1536, 512)])
+def test_non_power_of_two_block_counts(rd, D, p):
+    check_all(rd, 11, D, p, "f32", (400, 401, 402))
+
+
+def test_identity_layer_is_exact(rd):
+    """c_ii = delta, c_ij = 0: y = x and grad_x = g."""
+    B, D, p = 16, 1024, 256
+    q = D // p
+    c = np.zeros((q, q, p), dtype=np.float32)
+    for i in range(q):
+        c[i, i, 0] = 1.0
+    x = sample(410, (B, D), "f32")
+    c_hat = rd.circ_prepare(to_device(c, "f32"))
+    xd = to_device(x, "f32")
+    y = rd.circ_fwd(xd, c_hat, p)
+    gx, _ = rd.circ_bwd(xd, xd, c_hat, p)
+    torch.cuda.synchronize()
+    assert_parity(to_host_f64(y), x.exact, "f32", "identity y")
+    assert_parity(to_host_f64(gx), x.exact, "f32", "identity grad_x")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B", [1, 256])
+def test_config_d4096_p128(rd, B, dtype):
+    """D = 4096, p = 128 (q = 32), c ~ N(0, 1/D), x, g ~ N(0, 1), B in {1, 256}."""
+    check_all(rd, B, 4096, 128, dtype, (4, 5, 6))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("D,p,seed", [(4096, 1024, 7), (4096, 4096, 8), (1024, 1024, 9)])
+def test_config_block_size_extremes(rd, D, p, seed, dtype):
+    check_all(rd, 256, D, p, dtype, (seed, seed + 10, seed + 20))
+
+
+def test_config_adapter_stack_shape_sampled(rd):
+    """One adapter of the LLaMA2-7B-shaped stack at full size: D = 4096, p = 512,
+    4096 tokens, bf16. y and grad_x on the first and last 32 tokens, grad_c in full."""
+    B, D, p = 4096, 4096, 512
+    toks = np.r_[0:32, B - 32:B]
+    check_all(rd, B, D, p, "bf16", (300, 100, 200), tokens=toks)
+
+
+def test_grad_c_only_and_grad_x_only(rd):
+    B, D, p = 20, 1024, 128
+    c, x, g = make_layer(B, D, p, "f32", (500, 501, 502))
+    c_hat = rd.circ_prepare(to_device(c, "f32"))
+    xd, gd = to_device(x, "f32"), to_device(g, "f32")
+    gx, gc = rd.circ_bwd(gd, xd, c_hat, p, need_grad_c=False)
+    assert gc is None
+    gx2, gc2 = rd.circ_bwd(gd, xd, c_hat, p, need_grad_x=False)
+    assert gx2 is None
+    torch.cuda.synchronize()
+    gx_ref, gc_ref = oracle.circ_backward(g.exact, x.exact, c.exact)
+    assert_parity(to_host_f64(gx), gx_ref, "f32", "grad_x only")
+    assert_parity(to_host_f64(gc2), gc_ref, "f32", "grad_c only")
+
+
+def test_grad_c_overwrites_and_empty_batch(rd):
+    B, D, p = 8, 512, 64
+    c, x, g = make_layer(B, D, p, "f32", (510, 511, 512))
+    c_hat = rd.circ_prepare(to_device(c, "f32"))
+    xd, gd = to_device(x, "f32"), to_device(g, "f32")
+    gc = torch.full(c_hat.shape, 123.0, device="cuda")
+    rd.circ_bwd(gd, xd, c_hat, p, grad_c=gc, need_grad_x=False)
+    torch.cuda.synchronize()
+    _, gc_ref = oracle.circ_backward(g.exact, x.exact, c.exact)
+    assert_parity(to_host_f64(gc), gc_ref, "f32", "grad_c overwrite")
+    e = torch.empty((0, D), device="cuda")
+    gc.fill_(5.0)
+    rd.circ_bwd(e, e, c_hat, p, grad_c=gc, need_grad_x=False)
+    torch.cuda.synchronize()
+    assert torch.all(gc == 0)

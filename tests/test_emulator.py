@@ -1,0 +1,123 @@
+"""The kernels' per-thread rdFFT pass code, run on the host by the emulator, against
+the oracle: checks the pass plan, orbit indexing, bit reversal and butterflies of the
+CUDA path without a GPU."""
+import ctypes
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from conftest import ROOT
+from synthetic import bf16_bits_to_f64, round_to_bf16, sample
+
+PS = [2, 4, 8, 16, 32, 64, 128, 256, 512, 1024, 2048, 4096]
+
+
+@pytest.fixture(scope="module")
+def emu():
+    from block_circulant_layers_b200 import build
+    build.build_emulator()
+    L = ctypes.CDLL(os.path.join(ROOT, "block_circulant_layers_b200", "librdfft_hostemu.so"))
+    L.rdfft_emulate.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    L.rdfft_orbit_positions.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
+    L.rdfft_plan.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
+    return L
+
+
+def _rows_for(p):
+    # several CTAs and a ragged tail: a CTA owns 128/(p/32) rows (p >= 64) or 128 rows
+    per_cta = 128 if p <= 32 else max(1, 128 // (p // 32))
+    return 2 * per_cta + 1 if p < 2048 else 3
+
+
+@pytest.mark.parametrize("p", PS)
+def test_forward_fp32_matches_oracle(emu, p):
+    rows = _rows_for(p)
+    s = sample(1000 + p, (rows, p), "f32")
+    a = s.stored.copy()
+    assert emu.rdfft_emulate(a.ctypes.data, rows, p, 0, 0) == 0
+    ref = oracle.dft_packed(s.exact)
+    assert np.abs(a - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("p", PS)
+def test_inverse_fp32_matches_oracle(emu, p):
+    rows = _rows_for(p)
+    s = sample(2000 + p, (rows, p), "f32")
+    a = s.stored.copy()
+    assert emu.rdfft_emulate(a.ctypes.data, rows, p, 0, 1) == 0
+    ref = oracle.idft_packed(s.exact)
+    assert np.abs(a - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("p", [16, 512, 4096])
+def test_bf16_forward_and_inverse(emu, p):
+    rows = _rows_for(p)
+    s = sample(3000 + p, (rows, p), "bf16")
+    a = s.stored.copy()
+    assert emu.rdfft_emulate(a.ctypes.data, rows, p, 1, 0) == 0
+    ref = oracle.dft_packed(s.exact)
+    got = bf16_bits_to_f64(a)
+    assert np.all(np.abs(got - ref) <= 2e-2 * np.sqrt(np.mean(ref ** 2)))
+    b = a.copy()
+    assert emu.rdfft_emulate(b.ctypes.data, rows, p, 1, 1) == 0
+    ref_i = oracle.idft_packed(got)
+    assert np.all(np.abs(bf16_bits_to_f64(b) - ref_i) <= 2e-2 * np.sqrt(np.mean(ref_i ** 2)))
+
+
+def test_round_trip_and_empty(emu):
+    p, rows = 1024, 3
+    s = sample(4000, (rows, p), "f32")
+    a = s.stored.copy()
+    emu.rdfft_emulate(a.ctypes.data, rows, p, 0, 0)
+    emu.rdfft_emulate(a.ctypes.data, rows, p, 0, 1)
+    assert np.abs(a - s.stored).max() <= 1e-5 * np.abs(s.stored).max()
+    assert emu.rdfft_emulate(None, 0, p, 0, 0) == 0
+    assert emu.rdfft_emulate(a.ctypes.data, 1, 3, 0, 0) == 1
+
+
+def test_closed_form_delta(emu):
+    p = 512
+    a = np.zeros((1, p), dtype=np.float32)
+    a[0, 0] = 1.0
+    emu.rdfft_emulate(a.ctypes.data, 1, p, 0, 0)
+    want = np.zeros(p)
+    want[: p // 2 + 1] = 1.0
+    np.testing.assert_allclose(a[0], want, atol=1e-6)
+
+
+def test_bf16_store_rounding(emu):
+    """The store rounds fp32 once to nearest-even bf16 (checked on exact inputs)."""
+    p = 4
+    x = np.array([[1.0, 2.0 ** -8, 0.0, 0.0]])        # Y_0 = 1 + 2^-8: a tie -> 1.0
+    bits = round_to_bf16(x)
+    emu.rdfft_emulate(bits.ctypes.data, 1, p, 1, 0)
+    assert bf16_bits_to_f64(bits)[0, 0] == 1.0
+
+
+def test_proposition1_orbit_example(emu, golden):
+    """The kernels' orbit indexing reproduces the pages' four-element group example."""
+    (row,) = golden("prop1_groups.txt")
+    (M, k), group, (centre,), (texp,) = row
+    M, k, centre = int(M), int(k), int(centre)
+    group = [int(v) for v in group]
+    out = (ctypes.c_int * 4)()
+    emu.rdfft_orbit_positions(M // 2, k, 4, out)      # pass starting at H = M/2, residue k
+    pos = list(out)
+    assert pos == group
+    # symmetric about the centre: pairs (a1, b2) and (b1, a2)
+    assert pos[0] + pos[3] == 2 * centre and pos[1] + pos[2] == 2 * centre
+    assert int(texp) == k
+
+
+def test_pass_plan_covers_every_stage(emu):
+    s0 = (ctypes.c_int * 8)()
+    s1 = (ctypes.c_int * 8)()
+    for p in PS:
+        n = emu.rdfft_plan(p, s0, s1)
+        L = p.bit_length() - 1
+        assert s0[0] == 0 and s1[n - 1] == L
+        for i in range(1, n):
+            assert s0[i] == s1[i - 1]
+            assert s1[i] - s0[i] <= 4              # an orbit of <= 32 registers
