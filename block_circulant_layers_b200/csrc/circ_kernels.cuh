@@ -30,29 +30,45 @@
 
 namespace rdfft {
 
+// The layer kernels transform rows with 32 elements per thread (three passes at
+// p >= 1024): their registers are shared with the contraction's accumulators.
+template <int P>
+using LayerGeo = Geo<P, kEPT>;
+
 // ------------------------------------------------------------- tile row passes
+// Orbit pass K (tile -> tile) over tile rows [0, NR): every thread runs the generic
+// orbits of its rows, then the NR * NB merged orbits are spread one per thread.
+template <int P, int NT, int K, bool INV, typename T>
+__device__ __forceinline__ void tile_orbit_pass(float* tile, int NR) {
+  using G = LayerGeo<P>;
+  constexpr int TPR = G::TPR, RPR = NT / TPR;
+  constexpr int NB = PassShape<G, K>::NB;
+  const int v = threadIdx.x % TPR;
+  for (int r = threadIdx.x / TPR; r < NR; r += RPR)
+    generic_pass<G, K, INV, 0, 0>(tile, r, v, (T*)nullptr, false);
+  for (int mu = threadIdx.x; mu < NR * NB; mu += NT)
+    merged_orbit<G, K, INV, 0, 0>(tile, mu / NB, mu % NB, (T*)nullptr, false);
+}
+
 // Forward rdFFT of tile rows [0, NR): row r reads its input from src(r) (nullptr
 // means a row of zeros), the spectrum stays in the tile.
 template <int P, int NT, typename T, int K, typename SrcFn>
 __device__ __forceinline__ void fft_rows_rest(float* tile, int NR, SrcFn src) {
-  if constexpr (K < Plan<P>::NPASS) {
-    constexpr int TPR = Plan<P>::TPR, RPR = NT / TPR;
+  if constexpr (K < LayerGeo<P>::NPASS) {
     __syncthreads();
-    const int v = threadIdx.x % TPR;
-    for (int r = threadIdx.x / TPR; r < NR; r += RPR)
-      orbit_pass<P, K, false, 0, 0>(tile, r, v, (T*)nullptr, false);
+    tile_orbit_pass<P, NT, K, false, T>(tile, NR);
     fft_rows_rest<P, NT, T, K + 1>(tile, NR, src);
   }
 }
 
 template <int P, int NT, typename T, typename SrcFn>
 __device__ __forceinline__ void fft_rows(float* tile, int NR, SrcFn src) {
-  constexpr int TPR = Plan<P>::TPR, RPR = NT / TPR;
+  constexpr int TPR = LayerGeo<P>::TPR, RPR = NT / TPR;
   static_assert(NT % TPR == 0, "threads per CTA must cover whole rows");
   const int v = threadIdx.x % TPR;
   for (int r = threadIdx.x / TPR; r < NR; r += RPR) {
     const T* g = src(r);
-    fwd_pass0<P, T>(tile, r, v, g, g != nullptr);
+    fwd_pass0<LayerGeo<P>, T>(tile, r, v, g, g != nullptr);
   }
   fft_rows_rest<P, NT, T, 1>(tile, NR, src);
 }
@@ -61,18 +77,18 @@ __device__ __forceinline__ void fft_rows(float* tile, int NR, SrcFn src) {
 // written to dst(r) (nullptr: dropped).
 template <int P, int NT, typename T, int K, typename DstFn>
 __device__ __forceinline__ void ifft_rows(float* tile, int NR, DstFn dst) {
-  constexpr int NP = Plan<P>::NPASS;
-  constexpr int TPR = Plan<P>::TPR, RPR = NT / TPR;
+  constexpr int NP = LayerGeo<P>::NPASS;
+  constexpr int TPR = LayerGeo<P>::TPR, RPR = NT / TPR;
   if constexpr (K < NP) {
     if constexpr (K > 0) __syncthreads();
-    const int v = threadIdx.x % TPR;
-    for (int r = threadIdx.x / TPR; r < NR; r += RPR) {
-      if constexpr (K == NP - 1) {
+    if constexpr (K == NP - 1) {
+      const int v = threadIdx.x % TPR;
+      for (int r = threadIdx.x / TPR; r < NR; r += RPR) {
         T* g = dst(r);
-        inv_pass0<P, T>(tile, r, v, g, g != nullptr);
-      } else {
-        orbit_pass<P, NP - 1 - K, true, 0, 0>(tile, r, v, (T*)nullptr, false);
+        inv_pass0<LayerGeo<P>, T>(tile, r, v, g, g != nullptr);
       }
+    } else {
+      tile_orbit_pass<P, NT, NP - 1 - K, true, T>(tile, NR);
     }
     ifft_rows<P, NT, T, K + 1>(tile, NR, dst);
   }
@@ -96,6 +112,7 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
   const int64_t tok0 = (int64_t)blockIdx.x * TT;
   const int ntok = (int)((B - tok0) < TT ? (B - tok0) : TT);
   const int o0 = blockIdx.y * QI;            // first output block of this CTA
+  constexpr int RS = P + (P >> LayerGeo<P>::S);   // padded row stride of the tile
 
   // 1. rdFFT of the TT*q input rows (row r = t*q + b)
   fft_rows<P, NT, T>(tile, TT * q, [&](int r) -> const T* {
@@ -151,11 +168,12 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
         const float a2 = z ? 0.0f : (BWDX ? ci : -ci);
         const float a3 = z ? ci : cr;
         const float a4 = z ? 0.0f : (BWDX ? -ci : ci);
+        const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
-          const int row = t * q + j;
-          const float xr = tile[Swz<P>::at(row * P + k)];
-          const float xi = tile[Swz<P>::at(row * P + bin_im_slot<P>(k))];
+          const int rb = (t * q + j) * RS;
+          const float xr = tile[rb + kr];
+          const float xi = tile[rb + ki];
           acc_r[s][t] = fmaf(cr, xr, fmaf(a2, xi, acc_r[s][t]));
           acc_i[s][t] = fmaf(a3, xi, fmaf(a4, xr, acc_i[s][t]));
         }
@@ -170,11 +188,12 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
     const int pi = threadIdx.x + NT * s;
     const int ol = pi / HB, k = pi % HB;
     if (ol < QI) {
+      const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
-        const int row = t * QI + ol;
-        tile[Swz<P>::at(row * P + k)] = acc_r[s][t];
-        tile[Swz<P>::at(row * P + bin_im_slot<P>(k))] = acc_i[s][t];
+        const int rb = (t * QI + ol) * RS;
+        tile[rb + kr] = acc_r[s][t];
+        tile[rb + ki] = acc_i[s][t];
       }
     }
   }
@@ -202,6 +221,7 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   const int64_t tbeg = (int64_t)blockIdx.x * tok_per_cta;
   const int64_t tend = (tbeg + tok_per_cta < B) ? tbeg + tok_per_cta : B;
   const int nib = q / RI, njb = QJ / RJ;
+  constexpr int RS = P + (P >> LayerGeo<P>::S);   // padded row stride of the tile
   const int ngroups = HB * nib * njb;
 
   float s_r[NG][RI][RJ], s_i[NG][RI][RJ];
@@ -235,20 +255,20 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
         const int rest = gam / HB;
         const int ib = rest % nib, jb = rest / nib;
         const bool z = (k == 0);
-        const int kim = bin_im_slot<P>(k);
+        const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
         for (int t = 0; t < ntok; ++t) {
           float gr[RI], gi[RI];
 #pragma unroll
           for (int a = 0; a < RI; ++a) {
-            const int row = t * q + ib * RI + a;
-            gr[a] = tile[Swz<P>::at(row * P + k)];
-            gi[a] = tile[Swz<P>::at(row * P + kim)];
+            const int rb = (t * q + ib * RI + a) * RS;
+            gr[a] = tile[rb + kr];
+            gi[a] = tile[rb + ki];
           }
 #pragma unroll
           for (int b = 0; b < RJ; ++b) {
-            const int row = xrow0 + t * QJ + jb * RJ + b;
-            const float xr = tile[Swz<P>::at(row * P + k)];
-            const float xi = tile[Swz<P>::at(row * P + kim)];
+            const int rb = (xrow0 + t * QJ + jb * RJ + b) * RS;
+            const float xr = tile[rb + kr];
+            const float xi = tile[rb + ki];
             // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)
             const float xi_re = z ? 0.0f : xi;
             const float x_im = z ? xi : xr;
@@ -312,7 +332,7 @@ static cudaError_t launch_x_cfg(const void* in, const float* chat, void* out, in
   constexpr int QI_MAX = NS * NT / (P / 2);
   static_assert(QI_MAX >= 1, "slots must cover one block");
   const int QI = largest_divisor_leq(q, QI_MAX);
-  const size_t smem = sizeof(float) * (size_t)TT * q * P;
+  const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(TT * q);
   auto kern = k_circ_x<P, T, NT, TT, NS, BWDX>;
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
@@ -338,7 +358,8 @@ static cudaError_t launch_x_p(const void* in, const float* chat, void* out, int6
   } else {
     constexpr int NT = 128;
     constexpr int NS1 = (P / 2) / NT;                       // one output block per CTA
-    constexpr int NSM = NS1 * 4 <= 32 ? NS1 * 4 : 32;      // up to 4 (p=1024/2048) or 2 (p=4096)
+    // up to 4 output blocks (p = 1024), 2 (p = 2048, 4096); <= 32 slots, 16 at p = 2048
+    constexpr int NSM = P == 2048 ? 16 : (NS1 * 4 <= 32 ? NS1 * 4 : 32);
     if constexpr (P == 1024) {
       if (q == 1 && B >= 64) return launch_x_cfg<P, T, NT, 4, NS1, BWDX>(in, chat, out, B, q, s);
     }
@@ -350,7 +371,7 @@ template <int P, typename T, int NT, int TT, int NG, int RI, int RJ>
 static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B, int q, int QJ,
                           cudaStream_t s) {
   auto kern = k_circ_gc<P, T, NT, TT, NG, RI, RJ>;
-  const size_t smem = sizeof(float) * (size_t)TT * (q + QJ) * P;
+  const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(TT * (q + QJ));
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
   const int njgroups = q / QJ;

@@ -14,40 +14,48 @@
 namespace rdfft {
 namespace {
 
-template <int P, bool INV, int K, typename T>
-void emu_steps(float* tile, int rows_in_cta, int64_t row0, int64_t rows, T* data) {
-  if constexpr (K < Plan<P>::NPASS) {
-    constexpr int TPR = Plan<P>::TPR;
-    for (int tid = 0; tid < rows_in_cta * TPR; ++tid) {
-      const int lrow = tid / TPR, v = tid % TPR;
-      const int64_t row = row0 + lrow;
-      const bool active = row < rows;
-      T* g = data + (active ? row : 0) * P;
-      row_step<P, INV, K, T>(tile, lrow, v, g, active);
-    }
-    emu_steps<P, INV, K + 1, T>(tile, rows_in_cta, row0, rows, data);
+template <class G, bool INV, int K, int ROWS, typename T>
+void emu_steps(float* tile, int64_t row0, int64_t rows, T* data) {
+  if constexpr (K < G::NPASS) {
+    constexpr int TPR = G::TPR;
+    auto rowok = [&](int r) { return row0 + r < rows; };
+    auto rowptr = [&](int r) { return data + (row0 + r < rows ? row0 + r : (int64_t)0) * G::P; };
+    for (int tid = 0; tid < ROWS * TPR; ++tid)
+      row_step<G, INV, K, ROWS, T>(tile, tid / TPR, tid % TPR, rowptr, rowok);
+    emu_steps<G, INV, K + 1, ROWS, T>(tile, row0, rows, data);
   }
 }
 
+// Emulates the row transform of geometry G with ROWS rows per CTA.
+template <class G, int ROWS, bool INV, typename T>
+void emu_geo(T* data, int64_t rows) {
+  std::vector<float> tile(G::words(ROWS), 0.0f);
+  for (int64_t row0 = 0; row0 < rows; row0 += ROWS)
+    emu_steps<G, INV, 0, ROWS, T>(tile.data(), row0, rows, data);
+}
+
 template <int P, bool INV, typename T>
-void emu_rows(T* data, int64_t rows) {
-  constexpr int ROWS = RowTiling<P>::ROWS;
+void emu_rows(T* data, int64_t rows, int ept) {
   if constexpr (P <= 32) {
     for (int64_t r = 0; r < rows; ++r) row_small<P, INV, T>(data + r * P);
   } else {
-    std::vector<float> tile(ROWS * P, 0.0f);
-    for (int64_t row0 = 0; row0 < rows; row0 += ROWS)
-      emu_steps<P, INV, 0, T>(tile.data(), ROWS, row0, rows, data);
+    if (ept == 0) {
+      emu_geo<RowGeo<P>, RowTiling<P>::ROWS, INV, T>(data, rows);
+    } else {
+      // the layer kernels' geometry: 32 elements per thread, rows of a 128-thread CTA
+      using G = Geo<P, kEPT>;
+      emu_geo<G, (128 / G::TPR > 0 ? 128 / G::TPR : 1), INV, T>(data, rows);
+    }
   }
 }
 
 template <typename T>
-int emu_t(void* data, int64_t rows, int p, bool inv) {
+int emu_t(void* data, int64_t rows, int p, bool inv, int ept) {
   T* d = static_cast<T*>(data);
 #define RD_CASE(PP)                                   \
   case PP:                                            \
-    if (inv) emu_rows<PP, true, T>(d, rows);          \
-    else emu_rows<PP, false, T>(d, rows);             \
+    if (inv) emu_rows<PP, true, T>(d, rows, ept);     \
+    else emu_rows<PP, false, T>(d, rows, ept);        \
     return 0;
   switch (p) {
     RD_CASE(2) RD_CASE(4) RD_CASE(8) RD_CASE(16) RD_CASE(32) RD_CASE(64) RD_CASE(128)
@@ -65,8 +73,14 @@ extern "C" {
 // In-place emulated rdfft_fwd (inverse = 0) or rdfft_inv (inverse = 1) on host
 // memory; dtype 0 = fp32, 1 = bf16 bits. Returns 0, or 1 for an unsupported p.
 int rdfft_emulate(void* data, int64_t rows, int p, int dtype, int inverse) {
-  if (dtype == 0) return rdfft::emu_t<float>(data, rows, p, inverse != 0);
-  return rdfft::emu_t<rdfft::bf16_t>(data, rows, p, inverse != 0);
+  if (dtype == 0) return rdfft::emu_t<float>(data, rows, p, inverse != 0, 0);
+  return rdfft::emu_t<rdfft::bf16_t>(data, rows, p, inverse != 0, 0);
+}
+
+// The same with the layer kernels' row geometry (32 elements per thread).
+int rdfft_emulate_layer_rows(void* data, int64_t rows, int p, int dtype, int inverse) {
+  if (dtype == 0) return rdfft::emu_t<float>(data, rows, p, inverse != 0, 32);
+  return rdfft::emu_t<rdfft::bf16_t>(data, rows, p, inverse != 0, 32);
 }
 
 // Positions of the first n elements of the generic orbit with residue r of a pass
@@ -80,7 +94,7 @@ void rdfft_orbit_positions(int H, int r, int n, int* out) {
 int rdfft_plan(int p, int* s0, int* s1) {
   int L = 0;
   while ((1 << L) < p) ++L;
-  const int E = p < rdfft::kEPT ? p : rdfft::kEPT;
+  const int E = p < rdfft::ept_for(p) ? p : rdfft::ept_for(p);
   int e = 0;
   while ((1 << e) < E) ++e;
   int n = 0;

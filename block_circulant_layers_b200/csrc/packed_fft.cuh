@@ -51,7 +51,13 @@ namespace rdfft {
 
 // --------------------------------------------------------------------------- basics
 constexpr int kMaxP = 4096;
-constexpr int kEPT = 32;            // elements per thread in the multi-pass kernels
+constexpr int kEPT = 32;            // elements per thread of the multi-pass kernels, p <= 512
+
+// Elements per thread of the standalone transforms. 32 for every p: wider rows per
+// thread (64 at p = 1024/2048, 128 at p = 4096) save a shared-memory exchange but
+// measured slower on B200, the register cost lowering occupancy more than the saved
+// exchange gains.
+RD_HD constexpr int ept_for(int) { return kEPT; }
 
 RD_HD constexpr int ilog2(int n) { return n <= 1 ? 0 : 1 + ilog2(n >> 1); }
 
@@ -238,80 +244,81 @@ RD_HD void orbit_stages(float (&a)[E], int r) {
 }
 
 // ------------------------------------------------------------------------ plan
-// Pass 0 covers stages 1..e (blocks of E = 2^e); pass k >= 1 covers stages
-// s0+1..s1 with s0 = e + (k-1)(e-1), s1 = min(s0 + e - 1, L).
-template <int P>
-struct Plan {
+// Geometry of a row transform: row length P and elements per thread E (pass 0 runs
+// stages 1..e on contiguous blocks of E = 2^e; pass k >= 1 covers stages s0+1..s1
+// with s0 = e + (k-1)(e-1), s1 = min(s0 + e - 1, L)), and the padded tile layout:
+// word G (row lrow, element n at G = lrow*P + n) lives at G + (G >> S), one pad word
+// per 2^S words. S is chosen per geometry so that the 32 lanes of every pass-0
+// scatter and orbit gather/scatter fall in distinct banks (checked by a bank model),
+// and because every row/block base is a multiple of 2^S, each access is a per-thread
+// base register plus a compile-time offset.
+template <int P_, int EPT_>
+struct Geo {
+  static constexpr int P = P_;
   static_assert(P >= 2 && P <= kMaxP && (P & (P - 1)) == 0, "p must be a power of two in [2, 4096]");
   static constexpr int L = ilog2(P);
-  static constexpr int E = P < kEPT ? P : kEPT;
+  static constexpr int E = P < EPT_ ? P : EPT_;
   static constexpr int e = ilog2(E);
   static constexpr int TPR = P / E;               // threads per row
   static constexpr int LOG_TPR = ilog2(TPR);
   static constexpr int NPASS = (L <= e) ? 1 : 1 + (L - e + (e - 2)) / (e - 1);
   RD_HD static constexpr int s0(int k) { return e + (k - 1) * (e - 1); }
   RD_HD static constexpr int s1(int k) { return s0(k) + e - 1 < L ? s0(k) + e - 1 : L; }
+  static constexpr int S = (E <= 32) ? (P >= 4096 ? 7 : (P >= 2048 ? 6 : 5)) : e;
+  RD_HD static constexpr int at(int G) { return G + (G >> S); }
+  // words of a tile of `rows` rows (plus one spare word)
+  RD_HD static constexpr int words(int rows) { return at(rows * P) + 1; }
 };
 
-template <int P, int K>
+// The geometry of the standalone transforms: two passes for every p >= 64.
+template <int P>
+using RowGeo = Geo<P, ept_for(P)>;
+
+template <class G, int K>
 struct PassShape {
-  static constexpr int H = 1 << Plan<P>::s0(K);
-  static constexpr int LB = 1 << Plan<P>::s1(K);
+  static constexpr int H = 1 << G::s0(K);
+  static constexpr int LB = 1 << G::s1(K);
   static constexpr int UMAX = LB / H;
   static constexpr int N = 2 * UMAX;              // elements per orbit
-  static constexpr int C = Plan<P>::E / N;        // orbits per thread
+  static constexpr int C = G::E / N;              // orbits per thread
   static constexpr int HH = H / 2;                // orbits per block of LB
-};
-
-// Shared-memory swizzle of the row tile: XOR the low 5 bits of the word index with
-// a function of its higher bits, chosen per p so that the pass-0 scatter and the
-// orbit gathers/scatters of 32 lanes fall in distinct banks.
-template <int P>
-struct Swz {
-  static constexpr int A = P >= 4096 ? 2 : (P >= 2048 ? 1 : 0);
-  static constexpr int B = P >= 2048 ? 4 : -1;
-  RD_HD static int at(int G) {
-    const int g = G >> 5;
-    int f = (g >> A) & 31;
-    if (B >= 0) f ^= ((g >> (B < 0 ? 0 : B)) & 1) << 4;
-    return G ^ f;
-  }
+  static constexpr int NB = G::P / LB;            // blocks (merged orbits) per row
 };
 
 // ------------------------------------------------------------- per-thread passes
-// `tile` is the CTA's shared (or, in the emulator, host) fp32 row tile of ROWS*P
-// words; `lrow` the thread's row in the tile, `v` its index within the row's
-// TPR threads; `g` the row in global memory (valid only when `active`).
+// `tile` is the CTA's shared (or, in the emulator, host) fp32 row tile; `lrow` the
+// thread's row in the tile, `v` its index within the row's TPR threads; `g` the row
+// in global memory (valid only when `active`).
 
 // Forward pass 0: bit-reversed gather straight from global memory (coalesced:
 // lane v reads v + TPR*j'), stages 2..E in registers, scatter of block
 // t = bitrev(v) to the tile.
-template <int P, typename T>
+template <class G, typename T>
 RD_HD void fwd_pass0(float* tile, int lrow, int v, const T* g, bool active) {
-  using PL = Plan<P>;
-  float a[PL::E];
+  float a[G::E];
 #pragma unroll
-  for (int jp = 0; jp < PL::E; ++jp) a[bitrev(jp, PL::e)] = active ? ld(g + v + PL::TPR * jp) : 0.0f;
-  stages_contig<2, PL::E, PL::E, 0, false>(a);
-  const int t = bitrev(v, PL::LOG_TPR);
+  for (int jp = 0; jp < G::E; ++jp) a[bitrev(jp, G::e)] = active ? ld(g + v + G::TPR * jp) : 0.0f;
+  stages_contig<2, G::E, G::E, 0, false>(a);
+  const int t = bitrev(v, G::LOG_TPR);
+  float* dst = tile + G::at(lrow * G::P + t * G::E);    // block start, a multiple of 2^S
 #pragma unroll
-  for (int j = 0; j < PL::E; ++j) tile[Swz<P>::at(lrow * P + t * PL::E + j)] = a[j];
+  for (int j = 0; j < G::E; ++j) dst[j + (j >> G::S)] = a[j];
 }
 
 // Inverse pass 0 (the last inverse step): gather block t from the tile, inverse
 // stages E..2, scale by 1/P, scatter to global at the bit-reversed positions.
-template <int P, typename T>
+template <class G, typename T>
 RD_HD void inv_pass0(const float* tile, int lrow, int v, T* g, bool active) {
-  using PL = Plan<P>;
-  float a[PL::E];
-  const int t = bitrev(v, PL::LOG_TPR);
+  float a[G::E];
+  const int t = bitrev(v, G::LOG_TPR);
+  const float* src = tile + G::at(lrow * G::P + t * G::E);
 #pragma unroll
-  for (int j = 0; j < PL::E; ++j) a[j] = tile[Swz<P>::at(lrow * P + t * PL::E + j)];
-  stages_contig<2, PL::E, PL::E, 0, true>(a);
-  constexpr float scale = 1.0f / P;
+  for (int j = 0; j < G::E; ++j) a[j] = src[j + (j >> G::S)];
+  stages_contig<2, G::E, G::E, 0, true>(a);
+  constexpr float scale = 1.0f / G::P;
   if (active) {
 #pragma unroll
-    for (int j = 0; j < PL::E; ++j) g[v + PL::TPR * bitrev(j, PL::e)] = from_f32<T>(a[j] * scale);
+    for (int j = 0; j < G::E; ++j) g[v + G::TPR * bitrev(j, G::e)] = from_f32<T>(a[j] * scale);
   }
 }
 
@@ -324,57 +331,100 @@ RD_HD constexpr int orbit_pos(int H, int i, int r) {
   return (i & 1) ? ((i >> 1) + 1) * H - r : (i >> 1) * H + r;
 }
 
-// Slot CI of a middle/last pass K >= 1, then the following slots.
-// SRC/DST: 0 = tile, 1 = global row (natural order). Each of the thread's C orbits
-// is gathered, transformed and written back to the same positions, so a pass needs
-// no synchronisation inside itself.
-template <int P, int K, bool INV, int SRC, int DST, int CI, typename T, int E>
-RD_HD void orbit_slots(float (&a)[E], float* tile, int tb, int v, T* g, bool active) {
-  using PL = Plan<P>;
-  using S = PassShape<P, K>;
-  if constexpr (CI < S::C) {
-    constexpr int OFF = CI * S::N;
-    const int o = v + PL::TPR * CI;
-    const int beta = o / S::HH;
-    const int rho = o % S::HH;
-    const int base = beta * S::LB;
-    if (rho == 0) {
-      // merged orbit: positions base + l*H/2 form a packed real transform of N
-      // points whose first stage (M = 2) is already done.
-#pragma unroll
-      for (int l = 0; l < S::N; ++l) {
-        const int n = base + l * S::HH;
-        a[OFF + l] = SRC == 0 ? tile[Swz<P>::at(tb + n)] : (active ? ld(g + n) : 0.0f);
-      }
-      stages_contig<4, S::N, S::N, OFF, INV>(a);
-#pragma unroll
-      for (int l = 0; l < S::N; ++l) {
-        const int n = base + l * S::HH;
-        if (DST == 0) tile[Swz<P>::at(tb + n)] = a[OFF + l];
-        else if (active) g[n] = from_f32<T>(a[OFF + l]);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < S::N; ++i) {
-        const int n = base + orbit_pos(S::H, i, rho);
-        a[OFF + i] = SRC == 0 ? tile[Swz<P>::at(tb + n)] : (active ? ld(g + n) : 0.0f);
-      }
-      orbit_stages<S::H, S::UMAX, 2, OFF, INV>(a, rho);
-#pragma unroll
-      for (int i = 0; i < S::N; ++i) {
-        const int n = base + orbit_pos(S::H, i, rho);
-        if (DST == 0) tile[Swz<P>::at(tb + n)] = a[OFF + i];
-        else if (active) g[n] = from_f32<T>(a[OFF + i]);
-      }
-    }
-    orbit_slots<P, K, INV, SRC, DST, CI + 1>(a, tile, tb, v, g, active);
+// Orbit assignment of slot CI of pass K to thread v of its row: o = v + TPR*CI,
+// block beta = o / (H/2), residue rho = o % (H/2) (rho = 0: the merged orbit). In
+// pass 1 of rows with >= 32 threads and 16 residues per block, the two half-warps
+// take blocks NB/2 apart, so that their residues fall in opposite halves of the banks.
+template <class G, int K>
+RD_HD void orbit_of(int v, int CI, int& beta, int& rho) {
+  using S = PassShape<G, K>;
+  if constexpr (K == 1 && G::TPR >= 32 && S::HH == 16 && S::C == 1 && S::NB >= 2) {
+    const int lane = v & 31;
+    beta = (v >> 5) + (lane >> 4) * (S::NB / 2);
+    rho = lane & 15;
+  } else {
+    const int o = v + G::TPR * CI;
+    beta = o / S::HH;
+    rho = o % S::HH;
   }
 }
 
-template <int P, int K, bool INV, int SRC, int DST, typename T>
-RD_HD void orbit_pass(float* tile, int lrow, int v, T* g, bool active) {
-  float a[Plan<P>::E];
-  orbit_slots<P, K, INV, SRC, DST, 0>(a, tile, lrow * P, v, g, active);
+// Generic slots CI.. of a middle/last pass K >= 1 for thread v of the row at tile
+// offset tb (global row g). SRC/DST: 0 = tile, 1 = global row (natural order). Each
+// generic orbit is gathered, transformed and written back to the same positions, so
+// a pass needs no synchronisation inside itself. A slot whose residue is 0 (the
+// merged orbit) is skipped here: the merged orbits of all rows are done by
+// merged_orbit() below, one per thread, so that no warp runs both code paths.
+// Tile addresses: with R0 = row/block base (a multiple of 2^S) and c a compile-time
+// multiple of 32, the element at R0 + c + r sits at [R0 + (R0>>S) + r + (r>>S)] +
+// [c + (c>>S)] and the one at R0 + c - r (1 <= r) at [R0 + (R0>>S) - r - ((r-1)>>S)] +
+// [c + ((c-1)>>S)]: a per-thread base plus an immediate.
+template <class G, int K, bool INV, int SRC, int DST, int CI, typename T, int E>
+RD_HD void generic_slots(float (&a)[E], float* tile, int tb, int v, T* g, bool active) {
+  using S = PassShape<G, K>;
+  constexpr int SH = G::S;
+  if constexpr (CI < S::C) {
+    constexpr int OFF = CI * S::N;
+    int beta, rho;
+    orbit_of<G, K>(v, CI, beta, rho);
+    if (rho != 0) {
+      const int base = beta * S::LB;
+      float* tbase = tile + G::at(tb + base);
+      float* tp = tbase + rho + (rho >> SH);
+      float* tm = tbase - rho - ((rho - 1) >> SH);
+      T* gp = g + base + rho;
+      T* gm = g + base - rho;
+#pragma unroll
+      for (int m = 0; m < S::UMAX; ++m) {
+        const int cp = m * S::H, cm = (m + 1) * S::H;
+        a[OFF + 2 * m] = SRC == 0 ? tp[cp + (cp >> SH)] : (active ? ld(gp + cp) : 0.0f);
+        a[OFF + 2 * m + 1] = SRC == 0 ? tm[cm + ((cm - 1) >> SH)] : (active ? ld(gm + cm) : 0.0f);
+      }
+      orbit_stages<S::H, S::UMAX, 2, OFF, INV>(a, rho);
+#pragma unroll
+      for (int m = 0; m < S::UMAX; ++m) {
+        const int cp = m * S::H, cm = (m + 1) * S::H;
+        if (DST == 0) {
+          tp[cp + (cp >> SH)] = a[OFF + 2 * m];
+          tm[cm + ((cm - 1) >> SH)] = a[OFF + 2 * m + 1];
+        } else if (active) {
+          gp[cp] = from_f32<T>(a[OFF + 2 * m]);
+          gm[cm] = from_f32<T>(a[OFF + 2 * m + 1]);
+        }
+      }
+    }
+    generic_slots<G, K, INV, SRC, DST, CI + 1>(a, tile, tb, v, g, active);
+  }
+}
+
+template <class G, int K, bool INV, int SRC, int DST, typename T>
+RD_HD void generic_pass(float* tile, int lrow, int v, T* g, bool active) {
+  float a[G::E];
+  generic_slots<G, K, INV, SRC, DST, 0>(a, tile, lrow * G::P, v, g, active);
+}
+
+// The merged orbit of block beta of the row at tile row lrow in pass K: positions
+// base + l*H/2 (l < N) form a packed real transform of N points whose first stage
+// (M = 2) is already done; run its stages 4..N (or N..4 inverse).
+template <class G, int K, bool INV, int SRC, int DST, typename T>
+RD_HD void merged_orbit(float* tile, int lrow, int beta, T* g, bool active) {
+  using S = PassShape<G, K>;
+  constexpr int SH = G::S;
+  float a[S::N];
+  const int base = beta * S::LB;
+  float* tbase = tile + G::at(lrow * G::P + base);
+#pragma unroll
+  for (int l = 0; l < S::N; ++l) {
+    const int c = l * S::HH;
+    a[l] = SRC == 0 ? tbase[c + (c >> SH)] : (active ? ld(g + base + c) : 0.0f);
+  }
+  stages_contig<4, S::N, S::N, 0, INV>(a);
+#pragma unroll
+  for (int l = 0; l < S::N; ++l) {
+    const int c = l * S::HH;
+    if (DST == 0) tbase[c + (c >> SH)] = a[l];
+    else if (active) g[base + c] = from_f32<T>(a[l]);
+  }
 }
 
 }  // namespace rdfft

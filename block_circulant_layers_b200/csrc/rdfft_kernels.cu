@@ -12,12 +12,12 @@
 
 namespace rdfft {
 
-template <int P, bool INV, int K, typename T>
-__device__ __forceinline__ void run_steps(float* tile, int lrow, int v, T* g, bool active) {
-  if constexpr (K < Plan<P>::NPASS) {
+template <class G, bool INV, int K, int ROWS, typename T, typename RowPtr, typename RowOk>
+__device__ __forceinline__ void run_steps(float* tile, int lrow, int v, RowPtr rowptr, RowOk rowok) {
+  if constexpr (K < G::NPASS) {
     if constexpr (K > 0) __syncthreads();
-    row_step<P, INV, K, T>(tile, lrow, v, g, active);
-    run_steps<P, INV, K + 1, T>(tile, lrow, v, g, active);
+    row_step<G, INV, K, ROWS, T>(tile, lrow, v, rowptr, rowok);
+    run_steps<G, INV, K + 1, ROWS, T>(tile, lrow, v, rowptr, rowok);
   }
 }
 
@@ -29,14 +29,15 @@ k_rows(T* __restrict__ data, int64_t rows) {
     const int64_t row = (int64_t)blockIdx.x * ROWS + threadIdx.x;
     if (row < rows) row_small<P, INV, T>(data + row * P);
   } else {
-    constexpr int TPR = Plan<P>::TPR;
-    __shared__ float tile[ROWS * P];
+    using G = RowGeo<P>;
+    constexpr int TPR = G::TPR;
+    __shared__ float tile[G::words(ROWS)];
     const int lrow = threadIdx.x / TPR;
     const int v = threadIdx.x % TPR;
-    const int64_t row = (int64_t)blockIdx.x * ROWS + lrow;
-    const bool active = row < rows;
-    T* g = data + (active ? row : (int64_t)0) * P;
-    run_steps<P, INV, 0, T>(tile, lrow, v, g, active);
+    const int64_t row0 = (int64_t)blockIdx.x * ROWS;
+    auto rowok = [&](int r) { return row0 + r < rows; };
+    auto rowptr = [&](int r) { return data + (row0 + r < rows ? row0 + r : (int64_t)0) * P; };
+    run_steps<G, INV, 0, ROWS, T>(tile, lrow, v, rowptr, rowok);
   }
 }
 

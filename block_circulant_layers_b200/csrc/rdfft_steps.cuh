@@ -1,6 +1,6 @@
 // Per-thread steps of the standalone batched rdFFT / rdIFFT over rows of length P.
 //
-// A CTA owns ROWS consecutive rows and Plan<P>::TPR threads per row. Step k of the
+// A CTA owns ROWS consecutive rows and RowGeo<P>::TPR threads per row. Step k of the
 // forward transform runs pass k; step k of the inverse runs pass NPASS-1-k with the
 // inverse butterflies ("In-place IFFT design" on the paper-notes page of "Memory-
 // Efficient Training with In-Place FFT Implementation": the inverse reverses the
@@ -14,19 +14,29 @@
 
 namespace rdfft {
 
-template <int P, bool INV, int K, typename T>
-RD_HD void row_step(float* tile, int lrow, int v, T* g, bool active) {
-  constexpr int NP = Plan<P>::NPASS;
+// Step K for CTA thread tid = lrow * TPR + v. `rowptr(r)` gives the global row of
+// tile row r and `rowok(r)` whether it exists. Orbit passes run the thread's generic
+// orbits, then threads 0..NM-1 each run one merged orbit of the CTA's NM.
+template <class G, bool INV, int K, int ROWS, typename T, typename RowPtr, typename RowOk>
+RD_HD void row_step(float* tile, int lrow, int v, RowPtr rowptr, RowOk rowok) {
+  constexpr int NP = G::NPASS;
   static_assert(NP >= 2, "multi-pass rows only");
-  if constexpr (!INV) {
-    if constexpr (K == 0) fwd_pass0<P, T>(tile, lrow, v, g, active);
-    else if constexpr (K == NP - 1) orbit_pass<P, K, false, 0, 1>(tile, lrow, v, g, active);
-    else orbit_pass<P, K, false, 0, 0>(tile, lrow, v, g, active);
+  constexpr int PASS = INV ? NP - 1 - K : K;
+  T* g = rowptr(lrow);
+  const bool active = rowok(lrow);
+  if constexpr (PASS == 0) {
+    if constexpr (!INV) fwd_pass0<G, T>(tile, lrow, v, g, active);
+    else inv_pass0<G, T>(tile, lrow, v, g, active);
   } else {
-    constexpr int PASS = NP - 1 - K;
-    if constexpr (PASS == 0) inv_pass0<P, T>(tile, lrow, v, g, active);
-    else if constexpr (K == 0) orbit_pass<P, PASS, true, 1, 0>(tile, lrow, v, g, active);
-    else orbit_pass<P, PASS, true, 0, 0>(tile, lrow, v, g, active);
+    constexpr int SRC = (INV && K == 0) ? 1 : 0;
+    constexpr int DST = (!INV && K == NP - 1) ? 1 : 0;
+    generic_pass<G, PASS, INV, SRC, DST>(tile, lrow, v, g, active);
+    constexpr int NB = PassShape<G, PASS>::NB;
+    const int tid = lrow * G::TPR + v;
+    if (tid < ROWS * NB) {
+      const int mrow = tid / NB, beta = tid % NB;
+      merged_orbit<G, PASS, INV, SRC, DST>(tile, mrow, beta, rowptr(mrow), rowok(mrow));
+    }
   }
 }
 
@@ -51,11 +61,12 @@ RD_HD void row_small(T* g) {
   }
 }
 
-// Rows per CTA: 128 threads for the multi-pass rows, 128 rows for the small ones.
+// Rows per CTA: 32 threads (two rows) at p = 512, 128 threads otherwise (measured best
+// on B200 among 32..256 threads); 128 rows of one thread each for p <= 32.
 template <int P>
 struct RowTiling {
-  static constexpr int THREADS = 128;
-  static constexpr int ROWS = (P <= 32) ? THREADS : THREADS / Plan<P>::TPR;
+  static constexpr int THREADS = P == 512 ? 32 : 128;
+  static constexpr int ROWS = (P <= 32) ? THREADS : THREADS / RowGeo<P>::TPR;
 };
 
 }  // namespace rdfft

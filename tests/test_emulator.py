@@ -20,6 +20,7 @@ def emu():
     build.build_emulator()
     L = ctypes.CDLL(os.path.join(ROOT, "block_circulant_layers_b200", "librdfft_hostemu.so"))
     L.rdfft_emulate.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    L.rdfft_emulate_layer_rows.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     L.rdfft_orbit_positions.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
     L.rdfft_plan.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     return L
@@ -118,6 +119,22 @@ def test_pass_plan_covers_every_stage(emu):
         n = emu.rdfft_plan(p, s0, s1)
         L = p.bit_length() - 1
         assert s0[0] == 0 and s1[n - 1] == L
+        ept = min(p, 32)
+        assert s1[0] == ept.bit_length() - 1       # pass 0: blocks of ept elements
         for i in range(1, n):
             assert s0[i] == s1[i - 1]
-            assert s1[i] - s0[i] <= 4              # an orbit of <= 32 registers
+            assert 2 ** (s1[i] - s0[i] + 1) <= ept  # an orbit fits a thread's registers
+        assert n == (1 if p <= 32 else (2 if p <= 512 else 3))
+
+
+@pytest.mark.parametrize("p", [64, 128, 256, 512, 1024, 2048, 4096])
+def test_layer_row_geometry_matches_oracle(emu, p):
+    """The 32-element-per-thread geometry the layer kernels use (three passes at p >= 1024)."""
+    rows = 9 if p >= 1024 else 33
+    s = sample(5000 + p, (rows, p), "f32")
+    a = s.stored.copy()
+    assert emu.rdfft_emulate_layer_rows(a.ctypes.data, rows, p, 0, 0) == 0
+    ref = oracle.dft_packed(s.exact)
+    assert np.abs(a - ref).max() <= 1e-5 * np.abs(ref).max()
+    assert emu.rdfft_emulate_layer_rows(a.ctypes.data, rows, p, 0, 1) == 0
+    assert np.abs(a - s.exact).max() <= 1e-5 * np.abs(s.exact).max()
