@@ -461,7 +461,25 @@ def run_ours(args):
     st_t = time_graph(gst, 5, torch)
     layer["llama2_7b_shape_64_adapters_4096_tokens_per_step_tokens_s"] = round(B / st_t, 1)
     layer["llama2_7b_shape_ms_per_step"] = round(1e3 * st_t, 3)
-    del gst, xs, gs
+    del gst
+
+    # single-layer training-step peak memory at D = 4096 through the autograd module
+    # (in-place spectrum): parameter, its gradient, activations and their gradients
+    del xs, gs, cs, chs, gcs, ys, gxs
+    memory = {}
+    for Bm in (1, 256):
+        for pm in (128, 512, 1024, 4096):
+            torch.cuda.synchronize()
+            base = torch.cuda.memory_allocated(dev)
+            torch.cuda.reset_peak_memory_stats(dev)
+            lay = rd.BlockCirculantLinear(4096, pm, device=dev, generator=gen)
+            xm = torch.randn(Bm, 4096, device=dev, generator=gen).to(dt).requires_grad_(True)
+            ym = lay(xm)
+            ym.backward(torch.ones_like(ym))
+            torch.cuda.synchronize()
+            memory[f"B{Bm}_p{pm}_MB"] = round((torch.cuda.max_memory_allocated(dev) - base) / 1e6, 3)
+            del lay, xm, ym
+    layer["single_layer_train_step_peak_memory_d4096_bf16"] = memory
 
     # ---- CPU oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None

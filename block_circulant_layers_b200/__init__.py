@@ -12,14 +12,16 @@ Tensor functions (torch is used for device memory and the current stream):
     circ_fwd(x, c_hat, p, y=None)         y = W x
     circ_bwd(g, x, c_hat, p, grad_x=..., grad_c=...)
     circ_prepare(c)                       c_hat = packed rdfft_fwd of fp32 c
+    BlockCirculantLinear(D, p)            torch.nn.Module with autograd over the above
 Raw entry points on integer device pointers: ``lib`` (the ctypes handle).
 """
 from __future__ import annotations
 
 _EXPORTS = ("RDFFT_BF16", "RDFFT_F32", "RdfftError", "circ_bwd", "circ_fwd", "circ_prepare",
             "lib", "lib_path", "rdfft_fwd", "rdfft_inv")
+_LAYER = ("BlockCirculantLinear", "block_circulant")
 
-__all__ = list(_EXPORTS)
+__all__ = list(_EXPORTS + _LAYER)
 
 
 def __getattr__(name):
@@ -28,4 +30,7 @@ def __getattr__(name):
     if name in _EXPORTS:
         from . import _binding
         return getattr(_binding, name)
+    if name in _LAYER:
+        from . import layer
+        return getattr(layer, name)
     raise AttributeError(name)

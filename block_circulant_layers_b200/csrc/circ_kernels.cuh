@@ -73,25 +73,57 @@ __device__ __forceinline__ void fft_rows(float* tile, int NR, SrcFn src) {
   fft_rows_rest<P, NT, T, 1>(tile, NR, src);
 }
 
-// Inverse rdFFT of tile rows [0, NR) (the tile already synchronised); row r is
-// written to dst(r) (nullptr: dropped).
-template <int P, int NT, typename T, int K, typename DstFn>
-__device__ __forceinline__ void ifft_rows(float* tile, int NR, DstFn dst) {
-  constexpr int NP = LayerGeo<P>::NPASS;
-  constexpr int TPR = LayerGeo<P>::TPR, RPR = NT / TPR;
-  if constexpr (K < NP) {
-    if constexpr (K > 0) __syncthreads();
-    if constexpr (K == NP - 1) {
-      const int v = threadIdx.x % TPR;
-      for (int r = threadIdx.x / TPR; r < NR; r += RPR) {
-        T* g = dst(r);
-        inv_pass0<LayerGeo<P>, T>(tile, r, v, g, g != nullptr);
-      }
-    } else {
-      tile_orbit_pass<P, NT, NP - 1 - K, true, T>(tile, NR);
-    }
-    ifft_rows<P, NT, T, K + 1>(tile, NR, dst);
+// Last pass of a forward transform over tile rows [0, NR), written to global rows
+// dst(r) (nullptr: dropped) with the mirror epilogue: the Hartley form of the inverse.
+template <int P, int NT, typename T, typename DstFn>
+__device__ __forceinline__ void last_pass_mirror_to_global(float* tile, int NR, DstFn dst) {
+  using G = LayerGeo<P>;
+  constexpr int K = G::NPASS - 1;
+  constexpr int TPR = G::TPR, RPR = NT / TPR;
+  static_assert(PassShape<G, K>::NB == 1, "the last pass covers whole rows");
+  const int v = threadIdx.x % TPR;
+  for (int r = threadIdx.x / TPR; r < NR; r += RPR) {
+    T* g = dst(r);
+    generic_pass<G, K, false, 0, 1, T, 1>(tile, r, v, g, g != nullptr);
   }
+  for (int r = threadIdx.x; r < NR; r += NT) {
+    T* g = dst(r);
+    merged_orbit<G, K, false, 0, 1, T, 1>(tile, r, 0, g, g != nullptr);
+  }
+}
+
+template <int P, int NT, typename T, int K, typename DstFn>
+__device__ __forceinline__ void fwd_tile_passes_then_mirror(float* tile, int NR, DstFn dst) {
+  using G = LayerGeo<P>;
+  __syncthreads();
+  if constexpr (K < G::NPASS - 1) {
+    tile_orbit_pass<P, NT, K, false, T>(tile, NR);
+    fwd_tile_passes_then_mirror<P, NT, T, K + 1>(tile, NR, dst);
+  } else {
+    last_pass_mirror_to_global<P, NT, T>(tile, NR, dst);
+  }
+}
+
+// Inverse rdFFT of tile rows [0, NR) whose spectra were stored in mirrored form
+// (slot k = Re - Im, slot p-k = Re + Im of bin k; the caller has synchronised the
+// tile): by rdIFFT = (1/p) M rdFFT M, with M that mirror, this is a forward transform
+// of the tile rows with the mirror and the 1/p applied as the last pass writes row r
+// to dst(r). The forward butterflies cost 6 FP instructions per group against the
+// inverse's 8.
+template <int P, int NT, typename T, typename DstFn>
+__device__ __forceinline__ void ifft_rows_mirrored(float* tile, int NR, DstFn dst) {
+  using G = LayerGeo<P>;
+  constexpr int TPR = G::TPR, RPR = NT / TPR;
+  const int v = threadIdx.x % TPR;
+  // pass 0 in place in the tile: gather every row of a round, barrier, scatter
+  for (int r0 = 0; r0 < NR; r0 += RPR) {
+    const int r = r0 + threadIdx.x / TPR;
+    float a[G::E];
+    if (r < NR) fwd_pass0_load_tile<G>(a, v, tile + G::row_base(r));
+    __syncthreads();
+    if (r < NR) fwd_pass0_finish<G>(a, v, tile + G::row_base(r));
+  }
+  fwd_tile_passes_then_mirror<P, NT, T, 1>(tile, NR, dst);
 }
 
 // Packed-bin view of a row: bin 0 is the real pair (slot 0, slot p/2); bin k > 0 is
@@ -112,7 +144,6 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
   const int64_t tok0 = (int64_t)blockIdx.x * TT;
   const int ntok = (int)((B - tok0) < TT ? (B - tok0) : TT);
   const int o0 = blockIdx.y * QI;            // first output block of this CTA
-  constexpr int RS = P + (P >> LayerGeo<P>::S);   // padded row stride of the tile
 
   // 1. rdFFT of the TT*q input rows (row r = t*q + b)
   fft_rows<P, NT, T>(tile, TT * q, [&](int r) -> const T* {
@@ -171,7 +202,7 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
         const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
-          const int rb = (t * q + j) * RS;
+          const int rb = LayerGeo<P>::row_base(t * q + j);
           const float xr = tile[rb + kr];
           const float xi = tile[rb + ki];
           acc_r[s][t] = fmaf(cr, xr, fmaf(a2, xi, acc_r[s][t]));
@@ -191,16 +222,18 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
       const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
 #pragma unroll
       for (int t = 0; t < TT; ++t) {
-        const int rb = (t * QI + ol) * RS;
-        tile[rb + kr] = acc_r[s][t];
-        tile[rb + ki] = acc_i[s][t];
+        // stored mirrored (slot k = Re - Im, slot p-k = Re + Im) for the Hartley-form
+        // inverse below; bin 0 keeps its real pair
+        const int rb = LayerGeo<P>::row_base(t * QI + ol);
+        tile[rb + kr] = k == 0 ? acc_r[s][t] : acc_r[s][t] - acc_i[s][t];
+        tile[rb + ki] = k == 0 ? acc_i[s][t] : acc_r[s][t] + acc_i[s][t];
       }
     }
   }
   __syncthreads();
 
   // 4. rdIFFT of the TT*QI output rows straight to HBM
-  ifft_rows<P, NT, T, 0>(tile, TT * QI, [&](int r) -> T* {
+  ifft_rows_mirrored<P, NT, T>(tile, TT * QI, [&](int r) -> T* {
     const int t = r / QI, ol = r - t * QI;
     return t < ntok ? out + (tok0 + t) * (int64_t)D + (int64_t)(o0 + ol) * P : nullptr;
   });
@@ -221,7 +254,6 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   const int64_t tbeg = (int64_t)blockIdx.x * tok_per_cta;
   const int64_t tend = (tbeg + tok_per_cta < B) ? tbeg + tok_per_cta : B;
   const int nib = q / RI, njb = QJ / RJ;
-  constexpr int RS = P + (P >> LayerGeo<P>::S);   // padded row stride of the tile
   const int ngroups = HB * nib * njb;
 
   float s_r[NG][RI][RJ], s_i[NG][RI][RJ];
@@ -260,13 +292,13 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
           float gr[RI], gi[RI];
 #pragma unroll
           for (int a = 0; a < RI; ++a) {
-            const int rb = (t * q + ib * RI + a) * RS;
+            const int rb = LayerGeo<P>::row_base(t * q + ib * RI + a);
             gr[a] = tile[rb + kr];
             gi[a] = tile[rb + ki];
           }
 #pragma unroll
           for (int b = 0; b < RJ; ++b) {
-            const int rb = (xrow0 + t * QJ + jb * RJ + b) * RS;
+            const int rb = LayerGeo<P>::row_base(xrow0 + t * QJ + jb * RJ + b);
             const float xr = tile[rb + kr];
             const float xi = tile[rb + ki];
             // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)

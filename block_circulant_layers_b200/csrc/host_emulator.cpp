@@ -26,6 +26,26 @@ void emu_steps(float* tile, int64_t row0, int64_t rows, T* data) {
   }
 }
 
+// Forward orbit passes K.. of the Hartley-form inverse; the last one writes rows to
+// global memory with the mirror epilogue.
+template <class G, int K, typename T>
+void emu_hartley_rest(float* tile, int nr, T* rows) {
+  constexpr int TPR = G::TPR;
+  constexpr bool LAST = (K == G::NPASS - 1);
+  for (int tid = 0; tid < nr * TPR; ++tid) {
+    const int r = tid / TPR;
+    if constexpr (LAST) generic_pass<G, K, false, 0, 1, T, 1>(tile, r, tid % TPR, rows + (int64_t)r * G::P, true);
+    else generic_pass<G, K, false, 0, 0, T>(tile, r, tid % TPR, (T*)nullptr, false);
+  }
+  constexpr int NB = PassShape<G, K>::NB;
+  for (int mu = 0; mu < nr * NB; ++mu) {
+    const int r = mu / NB;
+    if constexpr (LAST) merged_orbit<G, K, false, 0, 1, T, 1>(tile, r, mu % NB, rows + (int64_t)r * G::P, true);
+    else merged_orbit<G, K, false, 0, 0, T>(tile, r, mu % NB, (T*)nullptr, false);
+  }
+  if constexpr (!LAST) emu_hartley_rest<G, K + 1, T>(tile, nr, rows);
+}
+
 // Emulates the row transform of geometry G with ROWS rows per CTA.
 template <class G, int ROWS, bool INV, typename T>
 void emu_geo(T* data, int64_t rows) {
@@ -46,6 +66,42 @@ void emu_rows(T* data, int64_t rows, int ept) {
       using G = Geo<P, kEPT>;
       emu_geo<G, (128 / G::TPR > 0 ? 128 / G::TPR : 1), INV, T>(data, rows);
     }
+  }
+}
+
+// The layer kernels' Hartley-form inverse of packed rows: mirror the spectrum (as
+// their contraction epilogue does), pass 0 from the tile, forward orbit passes, last
+// pass to global with the mirror epilogue. ROWS rows per emulated CTA.
+template <int P, typename T>
+void emu_hartley_inverse(T* data, int64_t rows) {
+  using G = Geo<P, kEPT>;
+  constexpr int TPR = G::TPR;
+  constexpr int ROWS = 128 / TPR > 0 ? 128 / TPR : 1;
+  std::vector<float> tile(G::words(ROWS), 0.0f);
+  std::vector<float> regs((size_t)ROWS * TPR * G::E);
+  for (int64_t row0 = 0; row0 < rows; row0 += ROWS) {
+    const int nr = (int)((rows - row0) < ROWS ? (rows - row0) : ROWS);
+    for (int r = 0; r < nr; ++r) {
+      const T* y = data + (row0 + r) * P;
+      float* trow = tile.data() + G::row_base(r);
+      trow[G::at(0)] = to_f32(y[0]);
+      trow[G::at(P / 2)] = to_f32(y[P / 2]);
+      for (int k = 1; k < P / 2; ++k) {
+        const float re = to_f32(y[k]), im = to_f32(y[P - k]);
+        trow[G::at(k)] = re - im;
+        trow[G::at(P - k)] = re + im;
+      }
+    }
+    // pass 0: every thread gathers, then every thread scatters
+    for (int tid = 0; tid < nr * TPR; ++tid) {
+      float(&a)[G::E] = *reinterpret_cast<float(*)[G::E]>(&regs[(size_t)tid * G::E]);
+      fwd_pass0_load_tile<G>(a, tid % TPR, tile.data() + G::row_base(tid / TPR));
+    }
+    for (int tid = 0; tid < nr * TPR; ++tid) {
+      float(&a)[G::E] = *reinterpret_cast<float(*)[G::E]>(&regs[(size_t)tid * G::E]);
+      fwd_pass0_finish<G>(a, tid % TPR, tile.data() + G::row_base(tid / TPR));
+    }
+    emu_hartley_rest<G, 1, T>(tile.data(), nr, data + row0 * P);
   }
 }
 
@@ -75,6 +131,21 @@ extern "C" {
 int rdfft_emulate(void* data, int64_t rows, int p, int dtype, int inverse) {
   if (dtype == 0) return rdfft::emu_t<float>(data, rows, p, inverse != 0, 0);
   return rdfft::emu_t<rdfft::bf16_t>(data, rows, p, inverse != 0, 0);
+}
+
+// The layer kernels' Hartley-form inverse (mirrored spectrum, forward transform,
+// mirror epilogue), in place on host rows; returns 1 for an unsupported p.
+int rdfft_emulate_hartley_inverse(void* data, int64_t rows, int p, int dtype) {
+#define RD_HCASE(PP)                                                                        \
+  case PP:                                                                                  \
+    if (dtype == 0) rdfft::emu_hartley_inverse<PP, float>(static_cast<float*>(data), rows); \
+    else rdfft::emu_hartley_inverse<PP, rdfft::bf16_t>(static_cast<rdfft::bf16_t*>(data), rows); \
+    return 0;
+  switch (p) {
+    RD_HCASE(64) RD_HCASE(128) RD_HCASE(256) RD_HCASE(512) RD_HCASE(1024) RD_HCASE(2048) RD_HCASE(4096)
+    default: return 1;
+  }
+#undef RD_HCASE
 }
 
 // The same with the layer kernels' row geometry (32 elements per thread).

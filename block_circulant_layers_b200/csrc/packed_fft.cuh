@@ -265,9 +265,16 @@ struct Geo {
   RD_HD static constexpr int s0(int k) { return e + (k - 1) * (e - 1); }
   RD_HD static constexpr int s1(int k) { return s0(k) + e - 1 < L ? s0(k) + e - 1 : L; }
   static constexpr int S = (E <= 32) ? (P >= 4096 ? 7 : (P >= 2048 ? 6 : 5)) : e;
-  RD_HD static constexpr int at(int G) { return G + (G >> S); }
+  // offset of element n within its row (n + one pad word per 2^S)
+  RD_HD static constexpr int at(int n) { return n + (n >> S); }
+  // Row r starts at r * RS plus one extra word per RW rows, RW being the rows that
+  // share a warp (32 / TPR, or 1): rows of one warp keep the bank pattern above, and
+  // the 32 rows whose merged orbits one warp processes get 32 distinct bank offsets.
+  static constexpr int RS = P + (P >> S);
+  static constexpr int RW = TPR < 32 ? 32 / TPR : 1;
+  RD_HD static constexpr int row_base(int r) { return r * RS + (RW > 1 ? r / RW : 0); }
   // words of a tile of `rows` rows (plus one spare word)
-  RD_HD static constexpr int words(int rows) { return at(rows * P) + 1; }
+  RD_HD static constexpr int words(int rows) { return row_base(rows) + 1; }
 };
 
 // The geometry of the standalone transforms: two passes for every p >= 64.
@@ -290,19 +297,43 @@ struct PassShape {
 // thread's row in the tile, `v` its index within the row's TPR threads; `g` the row
 // in global memory (valid only when `active`).
 
-// Forward pass 0: bit-reversed gather straight from global memory (coalesced:
-// lane v reads v + TPR*j'), stages 2..E in registers, scatter of block
-// t = bitrev(v) to the tile.
+// Forward pass 0: bit-reversed gather (lane v reads v + TPR*j', coalesced), stages
+// 2..E in registers, scatter of block t = bitrev(v) to the tile row.
+template <class G, typename T>
+RD_HD void fwd_pass0_load(float (&a)[G::E], int v, const T* g, bool active) {
+#pragma unroll
+  for (int jp = 0; jp < G::E; ++jp) a[bitrev(jp, G::e)] = active ? ld(g + v + G::TPR * jp) : 0.0f;
+}
+
+// The same gather from a tile row (for a transform whose input already sits in
+// shared memory); the caller puts a barrier between this and fwd_pass0_finish, as
+// the scatter overwrites positions other threads gather.
+// Element TPR*j' + v sits at [v + (v>>S)] + [TPR*j' + ((TPR*j')>>S)]: TPR*j' is a
+// multiple of TPR and, when TPR < 2^S, TPR*j' mod 2^S + v < 2^S.
+template <class G>
+RD_HD void fwd_pass0_load_tile(float (&a)[G::E], int v, const float* trow) {
+  const float* src = trow + v + (v >> G::S);
+#pragma unroll
+  for (int jp = 0; jp < G::E; ++jp) {
+    const int n = G::TPR * jp;
+    a[bitrev(jp, G::e)] = src[n + (n >> G::S)];
+  }
+}
+
+template <class G>
+RD_HD void fwd_pass0_finish(float (&a)[G::E], int v, float* trow) {
+  stages_contig<2, G::E, G::E, 0, false>(a);
+  const int t = bitrev(v, G::LOG_TPR);
+  float* dst = trow + G::at(t * G::E);          // block start, a multiple of 2^S
+#pragma unroll
+  for (int j = 0; j < G::E; ++j) dst[j + (j >> G::S)] = a[j];
+}
+
 template <class G, typename T>
 RD_HD void fwd_pass0(float* tile, int lrow, int v, const T* g, bool active) {
   float a[G::E];
-#pragma unroll
-  for (int jp = 0; jp < G::E; ++jp) a[bitrev(jp, G::e)] = active ? ld(g + v + G::TPR * jp) : 0.0f;
-  stages_contig<2, G::E, G::E, 0, false>(a);
-  const int t = bitrev(v, G::LOG_TPR);
-  float* dst = tile + G::at(lrow * G::P + t * G::E);    // block start, a multiple of 2^S
-#pragma unroll
-  for (int j = 0; j < G::E; ++j) dst[j + (j >> G::S)] = a[j];
+  fwd_pass0_load<G, T>(a, v, g, active);
+  fwd_pass0_finish<G>(a, v, tile + G::row_base(lrow));
 }
 
 // Inverse pass 0 (the last inverse step): gather block t from the tile, inverse
@@ -311,7 +342,7 @@ template <class G, typename T>
 RD_HD void inv_pass0(const float* tile, int lrow, int v, T* g, bool active) {
   float a[G::E];
   const int t = bitrev(v, G::LOG_TPR);
-  const float* src = tile + G::at(lrow * G::P + t * G::E);
+  const float* src = tile + G::row_base(lrow) + G::at(t * G::E);
 #pragma unroll
   for (int j = 0; j < G::E; ++j) a[j] = src[j + (j >> G::S)];
   stages_contig<2, G::E, G::E, 0, true>(a);
@@ -349,18 +380,30 @@ RD_HD void orbit_of(int v, int CI, int& beta, int& rho) {
   }
 }
 
-// Generic slots CI.. of a middle/last pass K >= 1 for thread v of the row at tile
-// offset tb (global row g). SRC/DST: 0 = tile, 1 = global row (natural order). Each
+// Mirror epilogue of the last pass (Hartley form of the inverse): with P the packed
+// forward transform of the mirrored spectrum, x_n = (P[n] - P[N-n]) / N and
+// x_{N-n} = (P[n] + P[N-n]) / N for 0 < n < N/2, x_0 = P[0] / N, x_{N/2} = P[N/2] / N.
+// `lo` and `hi` hold P at n < N/2 and N - n.
+RD_HD void mirror_pair(float& lo, float& hi, float scale) {
+  const float a = lo, b = hi;
+  lo = (a - b) * scale;
+  hi = (a + b) * scale;
+}
+
+// Generic slots CI.. of a middle/last pass K >= 1 for thread v of the tile row at
+// `trow` (global row g). SRC/DST: 0 = tile, 1 = global row (natural order). Each
 // generic orbit is gathered, transformed and written back to the same positions, so
 // a pass needs no synchronisation inside itself. A slot whose residue is 0 (the
 // merged orbit) is skipped here: the merged orbits of all rows are done by
 // merged_orbit() below, one per thread, so that no warp runs both code paths.
-// Tile addresses: with R0 = row/block base (a multiple of 2^S) and c a compile-time
+// EPI = 1 (last pass only, LB = P) applies the mirror epilogue before the store:
+// the mirror of element 2m (position mH + r) is element 2(U-1-m)+1, in the same orbit.
+// Tile addresses: with R0 = block base (a multiple of 2^S) and c a compile-time
 // multiple of 32, the element at R0 + c + r sits at [R0 + (R0>>S) + r + (r>>S)] +
 // [c + (c>>S)] and the one at R0 + c - r (1 <= r) at [R0 + (R0>>S) - r - ((r-1)>>S)] +
 // [c + ((c-1)>>S)]: a per-thread base plus an immediate.
-template <class G, int K, bool INV, int SRC, int DST, int CI, typename T, int E>
-RD_HD void generic_slots(float (&a)[E], float* tile, int tb, int v, T* g, bool active) {
+template <class G, int K, bool INV, int SRC, int DST, int EPI, int CI, typename T, int E>
+RD_HD void generic_slots(float (&a)[E], float* trow, int v, T* g, bool active) {
   using S = PassShape<G, K>;
   constexpr int SH = G::S;
   if constexpr (CI < S::C) {
@@ -369,7 +412,7 @@ RD_HD void generic_slots(float (&a)[E], float* tile, int tb, int v, T* g, bool a
     orbit_of<G, K>(v, CI, beta, rho);
     if (rho != 0) {
       const int base = beta * S::LB;
-      float* tbase = tile + G::at(tb + base);
+      float* tbase = trow + G::at(base);
       float* tp = tbase + rho + (rho >> SH);
       float* tm = tbase - rho - ((rho - 1) >> SH);
       T* gp = g + base + rho;
@@ -381,6 +424,16 @@ RD_HD void generic_slots(float (&a)[E], float* tile, int tb, int v, T* g, bool a
         a[OFF + 2 * m + 1] = SRC == 0 ? tm[cm + ((cm - 1) >> SH)] : (active ? ld(gm + cm) : 0.0f);
       }
       orbit_stages<S::H, S::UMAX, 2, OFF, INV>(a, rho);
+      if constexpr (EPI == 1) {
+        static_assert(S::LB == G::P && DST == 1, "mirror epilogue: last pass to global");
+        constexpr float scale = 1.0f / G::P;
+#pragma unroll
+        for (int m = 0; m < S::UMAX / 2; ++m)
+          mirror_pair(a[OFF + 2 * m], a[OFF + 2 * (S::UMAX - 1 - m) + 1], scale);
+#pragma unroll
+        for (int m = S::UMAX / 2; m < S::UMAX; ++m)
+          mirror_pair(a[OFF + 2 * (S::UMAX - 1 - m) + 1], a[OFF + 2 * m], scale);
+      }
 #pragma unroll
       for (int m = 0; m < S::UMAX; ++m) {
         const int cp = m * S::H, cm = (m + 1) * S::H;
@@ -393,32 +446,41 @@ RD_HD void generic_slots(float (&a)[E], float* tile, int tb, int v, T* g, bool a
         }
       }
     }
-    generic_slots<G, K, INV, SRC, DST, CI + 1>(a, tile, tb, v, g, active);
+    generic_slots<G, K, INV, SRC, DST, EPI, CI + 1>(a, trow, v, g, active);
   }
 }
 
-template <class G, int K, bool INV, int SRC, int DST, typename T>
+template <class G, int K, bool INV, int SRC, int DST, typename T, int EPI = 0>
 RD_HD void generic_pass(float* tile, int lrow, int v, T* g, bool active) {
   float a[G::E];
-  generic_slots<G, K, INV, SRC, DST, 0>(a, tile, lrow * G::P, v, g, active);
+  generic_slots<G, K, INV, SRC, DST, EPI, 0>(a, tile + G::row_base(lrow), v, g, active);
 }
 
 // The merged orbit of block beta of the row at tile row lrow in pass K: positions
 // base + l*H/2 (l < N) form a packed real transform of N points whose first stage
-// (M = 2) is already done; run its stages 4..N (or N..4 inverse).
-template <class G, int K, bool INV, int SRC, int DST, typename T>
+// (M = 2) is already done; run its stages 4..N (or N..4 inverse). EPI = 1 applies the
+// mirror epilogue (pairs l, N - l; l = 0 and N/2 are their own mirrors).
+template <class G, int K, bool INV, int SRC, int DST, typename T, int EPI = 0>
 RD_HD void merged_orbit(float* tile, int lrow, int beta, T* g, bool active) {
   using S = PassShape<G, K>;
   constexpr int SH = G::S;
   float a[S::N];
   const int base = beta * S::LB;
-  float* tbase = tile + G::at(lrow * G::P + base);
+  float* tbase = tile + G::row_base(lrow) + G::at(base);
 #pragma unroll
   for (int l = 0; l < S::N; ++l) {
     const int c = l * S::HH;
     a[l] = SRC == 0 ? tbase[c + (c >> SH)] : (active ? ld(g + base + c) : 0.0f);
   }
   stages_contig<4, S::N, S::N, 0, INV>(a);
+  if constexpr (EPI == 1) {
+    static_assert(S::LB == G::P && DST == 1, "mirror epilogue: last pass to global");
+    constexpr float scale = 1.0f / G::P;
+    a[0] *= scale;
+    a[S::N / 2] *= scale;
+#pragma unroll
+    for (int l = 1; l < S::N / 2; ++l) mirror_pair(a[l], a[S::N - l], scale);
+  }
 #pragma unroll
   for (int l = 0; l < S::N; ++l) {
     const int c = l * S::HH;

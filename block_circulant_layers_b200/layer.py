@@ -1,0 +1,92 @@
+"""PyTorch autograd module of the block-circulant linear layer over the C ABI.
+
+"Memory-Efficient Training with In-Place FFT Implementation" (paper-notes page,
+"Training strategy": the circulant structure replaces linear-layer weights, forward
+and backward run in place in the real domain, and the operator integrates with an
+autograd framework). The weight is D x D, made of q x q circulant blocks of size p
+given by c[i][j] (first columns, fp32). Every step of the computation runs in the
+library's kernels (rdfft_fwd / circ_fwd / circ_bwd / rdfft_inv); this file only
+marshals tensors.
+
+inplace_spectrum=True keeps no second copy of c: the spectrum c_hat is computed in
+c's own buffer (rdfft_fwd), used, and turned back into c (rdfft_inv) within the same
+forward or backward call. The round trip changes c by fp32 rounding only (relative
+error about 1e-7 per call). With inplace_spectrum=False a temporary c_hat is
+allocated by torch for each call instead.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from . import _binding as _b
+
+
+class _CirculantFn(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, c, p, inplace):
+        ctx.p = p
+        ctx.inplace = inplace
+        shape = x.shape
+        x2 = x.reshape(-1, shape[-1]).contiguous()
+        with torch.no_grad():
+            if inplace:
+                c_hat = _b.rdfft_fwd(c.data, p)
+            else:
+                c_hat = _b.circ_prepare(c.detach())
+            y = _b.circ_fwd(x2, c_hat, p)
+            if inplace:
+                _b.rdfft_inv(c.data, p)
+        ctx.save_for_backward(x2, c)
+        return y.reshape(shape)
+
+    @staticmethod
+    def backward(ctx, gy):
+        x2, c = ctx.saved_tensors
+        p = ctx.p
+        g2 = gy.reshape(-1, gy.shape[-1]).contiguous().to(x2.dtype)
+        need_x, need_c = ctx.needs_input_grad[0], ctx.needs_input_grad[1]
+        with torch.no_grad():
+            if ctx.inplace:
+                c_hat = _b.rdfft_fwd(c.data, p)
+            else:
+                c_hat = _b.circ_prepare(c.detach())
+            gx, gc = _b.circ_bwd(g2, x2, c_hat, p, need_grad_x=need_x, need_grad_c=need_c)
+            if ctx.inplace:
+                _b.rdfft_inv(c.data, p)
+        if gx is not None:
+            gx = gx.reshape(gy.shape)
+        return gx, gc, None, None
+
+
+def block_circulant(x: torch.Tensor, c: torch.Tensor, p: int, inplace_spectrum: bool = False) -> torch.Tensor:
+    """y = W(c) x over the last dimension of x (bf16 or fp32); c: (q, q, p) fp32."""
+    return _CirculantFn.apply(x, c, p, inplace_spectrum)
+
+
+class BlockCirculantLinear(torch.nn.Module):
+    """Linear layer D -> D whose weight is block circulant with block size p.
+
+    Parameters: c of shape (D/p, D/p, p), fp32, initialised i.i.d. N(0, 1/D) (the
+    synthetic initialisation used throughout this repository). Inputs may be bf16
+    or fp32; the arithmetic is fp32 and the output has the input's dtype.
+    """
+
+    def __init__(self, features: int, block: int, inplace_spectrum: bool = True, device=None,
+                 generator: torch.Generator | None = None):
+        super().__init__()
+        if block < 64 or block & (block - 1) or features % block:
+            raise ValueError("block must be a power of two >= 64 dividing features")
+        q = features // block
+        c = torch.randn(q, q, block, device=device, dtype=torch.float32, generator=generator)
+        self.c = torch.nn.Parameter(c / math.sqrt(features))
+        self.features = features
+        self.block = block
+        self.inplace_spectrum = inplace_spectrum
+
+    def forward(self, x: torch.Tensor) -> torch.Tensor:
+        return block_circulant(x, self.c, self.block, self.inplace_spectrum)
+
+    def extra_repr(self) -> str:
+        return f"features={self.features}, block={self.block}, inplace_spectrum={self.inplace_spectrum}"

@@ -21,6 +21,7 @@ def emu():
     L = ctypes.CDLL(os.path.join(ROOT, "block_circulant_layers_b200", "librdfft_hostemu.so"))
     L.rdfft_emulate.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     L.rdfft_emulate_layer_rows.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    L.rdfft_emulate_hartley_inverse.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_int]
     L.rdfft_orbit_positions.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int)]
     L.rdfft_plan.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int), ctypes.POINTER(ctypes.c_int)]
     return L
@@ -138,3 +139,15 @@ def test_layer_row_geometry_matches_oracle(emu, p):
     assert np.abs(a - ref).max() <= 1e-5 * np.abs(ref).max()
     assert emu.rdfft_emulate_layer_rows(a.ctypes.data, rows, p, 0, 1) == 0
     assert np.abs(a - s.exact).max() <= 1e-5 * np.abs(s.exact).max()
+
+
+@pytest.mark.parametrize("p", [64, 128, 256, 512, 1024, 2048, 4096])
+def test_hartley_form_inverse_matches_oracle(emu, p):
+    """The layer kernels' inverse: forward butterflies on the mirrored spectrum, then the
+    mirror and 1/p in the last pass (rdIFFT = (1/p) M rdFFT M)."""
+    rows = 9 if p >= 1024 else 33
+    s = sample(6000 + p, (rows, p), "f32")
+    a = s.stored.copy()
+    assert emu.rdfft_emulate_hartley_inverse(a.ctypes.data, rows, p, 0) == 0
+    ref = oracle.idft_packed(s.exact)
+    assert np.abs(a - ref).max() <= 1e-5 * np.abs(ref).max()

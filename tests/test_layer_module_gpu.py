@@ -1,0 +1,64 @@
+"""The autograd module over the C ABI: outputs and gradients against the oracle,
+and the in-place spectrum leaves the parameter as it was."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gpu_util import assert_parity, to_device, to_host_f64
+from synthetic import sample
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def rd():
+    if not torch.cuda.is_available():
+        pytest.fail("a CUDA GPU is required for the gpu tests")
+    import block_circulant_layers_b200 as rd
+    return rd
+
+
+@pytest.mark.parametrize("inplace", [True, False])
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_module_forward_backward(rd, inplace, dtype):
+    D, p, B = 1024, 128, 24
+    q = D // p
+    layer = rd.BlockCirculantLinear(D, p, inplace_spectrum=inplace, device="cuda")
+    c = sample(600, (q, q, p), "f32", sigma=1.0 / np.sqrt(D))
+    with torch.no_grad():
+        layer.c.copy_(to_device(c, "f32"))
+    x = sample(601, (3, B // 3, D), dtype)
+    g = sample(602, (3, B // 3, D), dtype)
+    xd = to_device(x, dtype).requires_grad_(True)
+    y = layer(xd)
+    y.backward(to_device(g, dtype))
+    torch.cuda.synchronize()
+    xe, ge = x.exact.reshape(B, D), g.exact.reshape(B, D)
+    assert_parity(to_host_f64(y).reshape(B, D), oracle.circ_forward(xe, c.exact), dtype, "module y")
+    gx_ref, gc_ref = oracle.circ_backward(ge, xe, c.exact)
+    assert_parity(to_host_f64(xd.grad).reshape(B, D), gx_ref, dtype, "module grad_x")
+    assert_parity(to_host_f64(layer.c.grad), gc_ref, dtype, "module grad_c")
+    # the parameter is unchanged up to the fp32 round trip of the in-place spectrum
+    diff = np.abs(to_host_f64(layer.c) - c.exact).max()
+    assert diff <= (1e-6 if inplace else 0.0) * np.abs(c.exact).max()
+
+
+def test_module_trains(rd):
+    """A few SGD steps on a least-squares target move the loss down."""
+    torch.manual_seed(0)
+    D, p = 512, 64
+    layer = rd.BlockCirculantLinear(D, p, device="cuda")
+    target = rd.BlockCirculantLinear(D, p, device="cuda")
+    x = torch.randn(64, D, device="cuda")
+    with torch.no_grad():
+        yt = target(x)
+    opt = torch.optim.SGD(layer.parameters(), lr=0.5)
+    losses = []
+    for _ in range(20):
+        opt.zero_grad()
+        loss = ((layer(x) - yt) ** 2).mean()
+        loss.backward()
+        opt.step()
+        losses.append(float(loss))
+    assert losses[-1] < 0.5 * losses[0]
