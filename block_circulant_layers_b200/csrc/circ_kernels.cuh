@@ -187,11 +187,15 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
       ci_c[s] = ci_n[s];
     }
     if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
+    // no guard on the slot here: a slot beyond the CTA's blocks has c = 0 (load_c), so
+    // its accumulators stay 0 and are never stored; without a branch, slots that share
+    // a bin (all of them when NT >= p/2) share the loads of X.
 #pragma unroll
-    for (int s = 0; s < NS; ++s) {
-      const int pi = threadIdx.x + NT * s;
-      const int ol = pi / HB, k = pi % HB;
-      if (ol < QI) {
+    for (int t = 0; t < TT; ++t) {
+      const int rb = LayerGeo<P>::row_base(t * q + j);
+#pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        const int k = (threadIdx.x + NT * s) % HB;
         const float cr = cr_c[s], ci = ci_c[s];
         // packed product: bin 0 multiplies the real pair component-wise, other bins
         // are complex products (conjugated c for grad_x)
@@ -199,15 +203,10 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
         const float a2 = z ? 0.0f : (BWDX ? ci : -ci);
         const float a3 = z ? ci : cr;
         const float a4 = z ? 0.0f : (BWDX ? -ci : ci);
-        const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
-#pragma unroll
-        for (int t = 0; t < TT; ++t) {
-          const int rb = LayerGeo<P>::row_base(t * q + j);
-          const float xr = tile[rb + kr];
-          const float xi = tile[rb + ki];
-          acc_r[s][t] = fmaf(cr, xr, fmaf(a2, xi, acc_r[s][t]));
-          acc_i[s][t] = fmaf(a3, xi, fmaf(a4, xr, acc_i[s][t]));
-        }
+        const float xr = tile[rb + LayerGeo<P>::at(k)];
+        const float xi = tile[rb + LayerGeo<P>::at(bin_im_slot<P>(k))];
+        acc_r[s][t] = fmaf(cr, xr, fmaf(a2, xi, acc_r[s][t]));
+        acc_i[s][t] = fmaf(a3, xi, fmaf(a4, xr, acc_i[s][t]));
       }
     }
   }
