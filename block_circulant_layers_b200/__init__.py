@@ -17,8 +17,8 @@ Raw entry points on integer device pointers: ``lib`` (the ctypes handle).
 """
 from __future__ import annotations
 
-_EXPORTS = ("RDFFT_BF16", "RDFFT_F32", "RdfftError", "circ_bwd", "circ_fwd", "circ_prepare",
-            "lib", "lib_path", "rdfft_fwd", "rdfft_inv")
+_EXPORTS = ("RDFFT_BF16", "RDFFT_F32", "RDFFT_ETIMEOUT", "RdfftError", "circ_bwd", "circ_fwd", "circ_prepare",
+            "lib", "lib_path", "rdfft_fwd", "rdfft_inv", "take_device_error", "selftest_wait_timeout")
 _LAYER = ("BlockCirculantLinear", "block_circulant")
 
 __all__ = list(_EXPORTS + _LAYER)

@@ -30,6 +30,12 @@ lib.rdfft_strerror.argtypes = [_int]
 lib.rdfft_strerror.restype = ctypes.c_char_p
 lib.rdfft_version.argtypes = []
 lib.rdfft_version.restype = _int
+lib.rdfft_take_device_error.argtypes = []
+lib.rdfft_take_device_error.restype = _int
+lib.rdfft_selftest_wait_timeout.argtypes = [_vp]
+lib.rdfft_selftest_wait_timeout.restype = _int
+
+RDFFT_ETIMEOUT = 7
 
 
 class RdfftError(RuntimeError):
@@ -141,3 +147,17 @@ def circ_bwd(g: torch.Tensor, x: torch.Tensor, c_hat: torch.Tensor, p: int,
         _check(lib.circ_bwd(g.data_ptr(), x.data_ptr(), c_hat.data_ptr(), gx_ptr, gc_ptr, B, D, p,
                             _dtype_code(x), _stream(x)), "circ_bwd")
     return (grad_x if need_grad_x else None), (grad_c if need_grad_c else None)
+
+
+def take_device_error() -> int:
+    """Device error state of the transform kernels since the last call (then cleared):
+    0, or RDFFT_ETIMEOUT when a bounded wait gave up. Synchronises with the device."""
+    code = lib.rdfft_take_device_error()
+    if code not in (0, RDFFT_ETIMEOUT):
+        raise RdfftError(code, "rdfft_take_device_error")
+    return code
+
+
+def selftest_wait_timeout() -> None:
+    """Enqueue the self-test kernel whose bounded wait runs out (about 1 ms)."""
+    _check(lib.rdfft_selftest_wait_timeout(torch.cuda.current_stream().cuda_stream), "rdfft_selftest_wait_timeout")

@@ -10,6 +10,12 @@ namespace rdfft {
 // rows of length p; dtype 0 = fp32, 1 = bf16. Arguments are already validated.
 cudaError_t launch_rows(void* data, int64_t rows, int p, int dtype, bool inverse, cudaStream_t s);
 
+// Reads and clears the error word of the rows kernels (bit 0: a bounded wait timed out).
+cudaError_t take_rows_device_error(unsigned int* flags);
+
+// Launches a kernel whose bounded wait must time out (self-test of the error path).
+cudaError_t launch_wait_selftest(cudaStream_t s);
+
 // Block-circulant layer forward: y = W x (see circ_fwd in rdfft.h).
 cudaError_t launch_circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p,
                             int dtype, cudaStream_t s);

@@ -103,12 +103,24 @@ const char* rdfft_strerror(int code) {
     case RDFFT_EALIGN: return "a pointer is not 16-byte aligned";
     case RDFFT_EDTYPE: return "dtype must be RDFFT_F32 (0) or RDFFT_BF16 (1)";
     case RDFFT_EOVERLAP: return "an output buffer overlaps an input buffer";
+    case RDFFT_ETIMEOUT: return "a kernel's bounded wait for its data timed out; its rows were not transformed";
     case RDFFT_ECUDA:
       snprintf(t_msg, sizeof(t_msg), "CUDA error while enqueuing: %s (%d)", cudaGetErrorString(t_last_cuda),
                (int)t_last_cuda);
       return t_msg;
     default: return "unknown rdfft error code";
   }
+}
+
+int rdfft_take_device_error(void) {
+  unsigned int flags = 0;
+  const cudaError_t e = rdfft::take_rows_device_error(&flags);
+  if (e != cudaSuccess) return finish(e);
+  return (flags & 1u) ? RDFFT_ETIMEOUT : RDFFT_OK;
+}
+
+int rdfft_selftest_wait_timeout(rdfft_stream_t stream) {
+  return finish(rdfft::launch_wait_selftest(reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int rdfft_version(void) { return 100; }

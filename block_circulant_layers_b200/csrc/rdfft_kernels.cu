@@ -7,6 +7,7 @@
 // tables, which stay in L1 / the constant cache.
 #include <cuda_runtime.h>
 
+#include "bulk_copy.cuh"
 #include "internal.h"
 #include "rdfft_steps.cuh"
 
@@ -21,6 +22,11 @@ __device__ __forceinline__ void run_steps(float* tile, int lrow, int v, RowPtr r
   }
 }
 
+// One CTA: ROWS consecutive rows. For p >= 64 the rows travel between HBM and a
+// padded shared staging buffer by bulk copies (the TMA engine, no per-element load or
+// store instructions), and the passes read their first input from and write their
+// last output to that buffer. The pad (64 bytes per row) puts the two rows that share
+// a warp at p = 512 in opposite halves of the banks.
 template <int P, bool INV, typename T>
 __global__ void __launch_bounds__(RowTiling<P>::THREADS)
 k_rows(T* __restrict__ data, int64_t rows) {
@@ -31,14 +37,58 @@ k_rows(T* __restrict__ data, int64_t rows) {
   } else {
     using G = RowGeo<P>;
     constexpr int TPR = G::TPR;
+    constexpr int RAW_ROW = P * (int)sizeof(T);
+    constexpr int RAW_STRIDE = RAW_ROW + 64;
+    __shared__ __align__(128) unsigned char raw[ROWS * RAW_STRIDE];
     __shared__ float tile[G::words(ROWS)];
+    __shared__ __align__(8) uint64_t mbar;
+    const int64_t row0 = (int64_t)blockIdx.x * ROWS;
+    const int nr = (int)((rows - row0) < ROWS ? (rows - row0) : ROWS);
+    if (threadIdx.x == 0) {
+      mbar_init(&mbar, 1);
+      mbar_arrive_expect_tx(&mbar, (unsigned)(nr * RAW_ROW));
+      for (int r = 0; r < nr; ++r) bulk_load(raw + r * RAW_STRIDE, data + (row0 + r) * P, RAW_ROW, &mbar);
+    }
+    __syncthreads();                                  // the barrier exists before anyone waits
+    const bool arrived = mbar_wait_bounded(&mbar, 0);
+    if (!__syncthreads_and(arrived)) {
+      mbar_wait_bounded(&mbar, 0);                    // give copies in flight a last chance
+      return;
+    }
     const int lrow = threadIdx.x / TPR;
     const int v = threadIdx.x % TPR;
-    const int64_t row0 = (int64_t)blockIdx.x * ROWS;
-    auto rowok = [&](int r) { return row0 + r < rows; };
-    auto rowptr = [&](int r) { return data + (row0 + r < rows ? row0 + r : (int64_t)0) * P; };
+    auto rowok = [&](int r) { return r < nr; };
+    auto rowptr = [&](int r) { return reinterpret_cast<T*>(raw + r * RAW_STRIDE); };
     run_steps<G, INV, 0, ROWS, T>(tile, lrow, v, rowptr, rowok);
+    fence_smem_to_async();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      for (int r = 0; r < nr; ++r) bulk_store(data + (row0 + r) * P, raw + r * RAW_STRIDE, RAW_ROW);
+      bulk_commit();
+      bulk_wait_all();
+    }
   }
+}
+
+// Self-test of the bounded wait: an mbarrier that expects 16 bytes nobody sends.
+__global__ void k_wait_selftest(long long limit_cycles) {
+  __shared__ __align__(8) uint64_t mbar;
+  mbar_init(&mbar, 1);
+  mbar_arrive_expect_tx(&mbar, 16);
+  mbar_wait_bounded(&mbar, 0, limit_cycles);
+}
+
+cudaError_t take_rows_device_error(unsigned int* flags) {
+  unsigned int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  *flags = v;
+  return e;
+}
+
+cudaError_t launch_wait_selftest(cudaStream_t s) {
+  k_wait_selftest<<<1, 1, 0, s>>>(2000000LL);          // about a millisecond
+  return cudaGetLastError();
 }
 
 template <int P, typename T>

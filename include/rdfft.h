@@ -60,7 +60,8 @@ enum {
   RDFFT_EALIGN = 3,   /* a pointer is not 16-byte aligned */
   RDFFT_EDTYPE = 4,   /* dtype is neither RDFFT_F32 nor RDFFT_BF16 */
   RDFFT_ECUDA = 5,    /* a CUDA call failed while enqueuing work */
-  RDFFT_EOVERLAP = 6  /* an output buffer overlaps an input buffer it may not alias */
+  RDFFT_EOVERLAP = 6, /* an output buffer overlaps an input buffer it may not alias */
+  RDFFT_ETIMEOUT = 7  /* reported by rdfft_take_device_error(): a bounded device wait gave up */
 };
 
 /* Largest feature size D accepted by circ_fwd / circ_bwd. */
@@ -128,6 +129,26 @@ int circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p
  */
 int circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
              int64_t B, int D, int p, int dtype, rdfft_stream_t stream);
+
+/*
+ * rdfft_take_device_error -- the device error state of the transform kernels, then cleared.
+ * No page has this; it is the library's failure detection. The row kernels move rows
+ * with bulk copies and wait for them on a barrier with a bounded wait (about one
+ * second): a wait that gives up leaves its rows unchanged, and records the event in a
+ * word of the module's device memory instead of hanging the GPU. This call reads and
+ * clears that word for the current device. It synchronises with the device (a
+ * cudaMemcpyFromSymbol), so call it between steps, not inside a captured graph.
+ * Returns RDFFT_OK, RDFFT_ETIMEOUT, or RDFFT_ECUDA.
+ */
+int rdfft_take_device_error(void);
+
+/*
+ * rdfft_selftest_wait_timeout -- enqueues a one-thread kernel whose bounded wait (about
+ * one millisecond) is made to run out, on a barrier that expects bytes nobody sends.
+ * No page has this; it lets a test check the failure path without any fault: after it
+ * completes, rdfft_take_device_error() returns RDFFT_ETIMEOUT.
+ */
+int rdfft_selftest_wait_timeout(rdfft_stream_t stream);
 
 /* Human-readable message for a return code (per host thread for RDFFT_ECUDA). */
 const char* rdfft_strerror(int code);

@@ -13,7 +13,7 @@ from conftest import ROOT
 PKG = os.path.join(ROOT, "block_circulant_layers_b200")
 HEADER = os.path.join(ROOT, "include", "rdfft.h")
 
-OK, EINVAL, ENULL, EALIGN, EDTYPE, ECUDA, EOVERLAP = range(7)
+OK, EINVAL, ENULL, EALIGN, EDTYPE, ECUDA, EOVERLAP, ETIMEOUT = range(8)
 F32, BF16 = 0, 1
 
 
@@ -40,7 +40,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for n in ("rdfft_fwd", "rdfft_inv", "circ_fwd", "circ_bwd", "rdfft_strerror", "rdfft_version"):
+    for n in ("rdfft_fwd", "rdfft_inv", "circ_fwd", "circ_bwd", "rdfft_strerror", "rdfft_version",
+              "rdfft_take_device_error", "rdfft_selftest_wait_timeout"):
         assert n in names
 
 
@@ -56,7 +57,7 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_version_and_messages(lib):
     assert lib.rdfft_version() >= 100
-    for code in range(7):
+    for code in range(8):
         assert lib.rdfft_strerror(code)
     assert b"unknown" in lib.rdfft_strerror(99)
 

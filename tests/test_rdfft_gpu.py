@@ -134,3 +134,24 @@ def test_errors_raise(rd):
         rd.rdfft_fwd(t, 3)
     with pytest.raises(TypeError):
         rd.rdfft_fwd(torch.zeros(512, device="cuda", dtype=torch.float16), 512)
+
+
+def test_bounded_wait_error_path(rd):
+    """No wait times out in normal use; the self-test's wait runs out and is reported,
+    once, without any fault."""
+    p = 4096
+    t = torch.randn(300, p, device="cuda").to(torch.bfloat16)
+    rd.rdfft_fwd(t, p)
+    rd.rdfft_inv(t, p)
+    torch.cuda.synchronize()
+    assert rd.take_device_error() == 0
+    rd.selftest_wait_timeout()
+    torch.cuda.synchronize()
+    assert rd.take_device_error() == rd.RDFFT_ETIMEOUT
+    assert rd.take_device_error() == 0
+    # the transforms still work afterwards
+    s = sample(33_000, (5, p), "f32")
+    x = to_device(s, "f32")
+    rd.rdfft_fwd(x, p)
+    torch.cuda.synchronize()
+    assert_parity(to_host_f64(x), oracle.dft_packed(s.exact), "f32", "after self-test")
