@@ -18,6 +18,12 @@ no reordering beyond the definition):
   layer as a dense D x D matrix built from its q x q circulant blocks (paper-notes
   page, method section, "Circulant matrix training adaptation"), with grad_x the
   transposed product and grad_c the chain rule through the matrix entries.
+* packed_to_rfft / rfft_to_packed -- the cast between a packed row and its explicit
+  complex bins Y_0..Y_{p/2} (summary page, "Limitations").
+* dft2_packed / unpack2_spectrum / idft2_packed -- the 2-D real DFT of an R x C
+  image by its definition (two DFT matrices), written into the per-axis packed
+  layout documented in dft2_packed (paper-notes page, "Limitations and outlook"
+  leaves 2-D open; that layout is the reading taken).
 
 Every function here is pinned by tests/test_oracle_pins.py against closed forms,
 invariants, a library FFT on the special cases that reduce to it, hand values and
@@ -30,4 +36,10 @@ from .rdfft_oracle import (  # noqa: F401
     circulant_matrix,
     circ_forward,
     circ_backward,
+    packed_to_rfft,
+    rfft_to_packed,
+    dft2_full,
+    dft2_packed,
+    unpack2_spectrum,
+    idft2_packed,
 )

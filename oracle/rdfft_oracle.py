@@ -142,3 +142,118 @@ def circ_backward(g: np.ndarray, x: np.ndarray, c: np.ndarray):
         m = (n - k) % p
         grad_c[:, :, k] = dW[:, n, :, m].sum(axis=0)   # advanced dims first: (p, q, q)
     return grad_x, grad_c
+
+
+# ------------------------------------------------------ explicit complex spectrum
+def packed_to_rfft(y: np.ndarray) -> np.ndarray:
+    """Bins Y_0..Y_{p/2} (complex128, shape (..., p/2 + 1)) of packed rows y.
+
+    The explicit complex spectrum that the packed layout encodes implicitly
+    ("Memory-Efficient Training with In-Place FFT Implementation", summary page,
+    "Limitations": reaching it needs a cast out of the in-place buffer, since p
+    reals become p/2 + 1 complex values). Bins 0 and p/2 have zero imaginary part.
+    """
+    Y = unpack_spectrum(y)
+    return Y[..., : y.shape[-1] // 2 + 1].copy()
+
+
+def rfft_to_packed(z: np.ndarray) -> np.ndarray:
+    """Packed rows (float64, shape (..., p)) of bins z = Y_0..Y_{p/2}, p = 2 (n - 1).
+
+    Inverse of packed_to_rfft on spectra of real rows: slot k takes Re Y_k and slot
+    p - k takes Im Y_k for 0 < k < p/2; the imaginary parts of Y_0 and Y_{p/2}
+    (zero for a real row) are not stored.
+    """
+    z = np.asarray(z, dtype=np.complex128)
+    p = 2 * (z.shape[-1] - 1)
+    _check_p(p)
+    h = p // 2
+    out = np.empty(z.shape[:-1] + (p,), dtype=np.float64)
+    out[..., : h + 1] = z.real
+    for k in range(1, h):
+        out[..., p - k] = z[..., k].imag
+    return out
+
+
+# ------------------------------------------------------------------- 2-D rdFFT
+def _dft_matrix(n: int) -> np.ndarray:
+    """F[k, m] = exp(-2 pi i (k m mod n) / n), complex128."""
+    cos, sin = _dft_cos_sin(n)
+    return cos - 1j * sin
+
+
+def dft2_full(x: np.ndarray) -> np.ndarray:
+    """2-D DFT Y[k1, k2] = sum_{r, c} x[r, c] e^{-2 pi i (k1 r / R + k2 c / C)} of the
+    last two axes of real x (shape (..., R, C)), complex128, by the definition."""
+    x = np.asarray(x, dtype=np.float64)
+    R, C = x.shape[-2:]
+    return _dft_matrix(R) @ x @ _dft_matrix(C).T
+
+
+def dft2_packed(x: np.ndarray) -> np.ndarray:
+    """Packed 2-D real DFT of the last two axes of x (shape (..., R, C)), float64.
+
+    The pages leave the 2-D transform open (paper-notes page, "Limitations and
+    outlook": only 1-D is done). The reading taken is the packed layout applied per
+    axis, so that every slot holds one real number of the spectrum, as in 1-D:
+      * columns 0 < k2 < C/2: slot [k1, k2] = Re Y[k1, k2] and slot [k1, C - k2] =
+        Im Y[k1, k2] for every row k1 < R;
+      * columns k2 in {0, C/2}: Y[., k2] is the spectrum of a real sequence
+        (conjugate symmetric in k1), stored in the 1-D packed layout down the
+        column: [0] = Y[0, k2], [R/2] = Y[R/2, k2], [k1] = Re Y[k1, k2],
+        [R - k1] = Im Y[k1, k2] for 0 < k1 < R/2.
+    Every value of the non-redundant half-spectrum appears exactly once.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    R, C = x.shape[-2:]
+    _check_p(R)
+    _check_p(C)
+    Y = dft2_full(x)
+    out = np.empty_like(x)
+    h = C // 2
+    for k2 in range(1, h):
+        out[..., :, k2] = Y[..., :, k2].real
+        out[..., :, C - k2] = Y[..., :, k2].imag
+    for k2 in (0, h):
+        col = Y[..., :, k2]
+        out[..., 0, k2] = col[..., 0].real
+        out[..., R // 2, k2] = col[..., R // 2].real
+        for k1 in range(1, R // 2):
+            out[..., k1, k2] = col[..., k1].real
+            out[..., R - k1, k2] = col[..., k1].imag
+    return out
+
+
+def unpack2_spectrum(y: np.ndarray) -> np.ndarray:
+    """Full 2-D spectrum Y[k1, k2] (complex128, shape (..., R, C)) of packed y.
+
+    Reads dft2_packed's layout and fills the rest by the symmetry of a real
+    image's spectrum, Y[(R - k1) mod R, (C - k2) mod C] = conj(Y[k1, k2]).
+    """
+    y = np.asarray(y, dtype=np.float64)
+    R, C = y.shape[-2:]
+    _check_p(R)
+    _check_p(C)
+    h = C // 2
+    Y = np.zeros(y.shape, dtype=np.complex128)
+    for k2 in range(1, h):
+        Y[..., :, k2] = y[..., :, k2] + 1j * y[..., :, C - k2]
+    for k2 in (0, h):
+        Y[..., 0, k2] = y[..., 0, k2]
+        Y[..., R // 2, k2] = y[..., R // 2, k2]
+        for k1 in range(1, R // 2):
+            Y[..., k1, k2] = y[..., k1, k2] + 1j * y[..., R - k1, k2]
+            Y[..., R - k1, k2] = y[..., k1, k2] - 1j * y[..., R - k1, k2]
+    k1 = np.arange(R)
+    for k2 in range(h + 1, C):
+        Y[..., :, k2] = np.conj(Y[..., (R - k1) % R, C - k2])
+    return Y
+
+
+def idft2_packed(y: np.ndarray) -> np.ndarray:
+    """Inverse of dft2_packed: x[r, c] = (1/(R C)) sum_{k1, k2} Y[k1, k2]
+    e^{+2 pi i (k1 r / R + k2 c / C)}, float64 (the real part of the sum)."""
+    Y = unpack2_spectrum(y)
+    R, C = Y.shape[-2:]
+    x = np.conj(_dft_matrix(R)) @ Y @ np.conj(_dft_matrix(C)).T
+    return x.real / (R * C)
