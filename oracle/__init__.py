@@ -23,7 +23,8 @@ no reordering beyond the definition):
 * dft2_packed / unpack2_spectrum / idft2_packed -- the 2-D real DFT of an R x C
   image by its definition (two DFT matrices), written into the per-axis packed
   layout documented in dft2_packed (paper-notes page, "Limitations and outlook"
-  leaves 2-D open; that layout is the reading taken).
+  leaves 2-D open; that layout is the reading taken); dft2_packed_at gives single
+  slots of it by the definition, for images too large for the matrix form.
 
 Every function here is pinned by tests/test_oracle_pins.py against closed forms,
 invariants, a library FFT on the special cases that reduce to it, hand values and
@@ -40,6 +41,7 @@ from .rdfft_oracle import (  # noqa: F401
     rfft_to_packed,
     dft2_full,
     dft2_packed,
+    dft2_packed_at,
     unpack2_spectrum,
     idft2_packed,
 )

@@ -257,3 +257,32 @@ def idft2_packed(y: np.ndarray) -> np.ndarray:
     R, C = Y.shape[-2:]
     x = np.conj(_dft_matrix(R)) @ Y @ np.conj(_dft_matrix(C)).T
     return x.real / (R * C)
+
+
+def dft2_packed_at(x: np.ndarray, slots) -> np.ndarray:
+    """Values of the packed 2-D spectrum of one image x (R x C) at the given slots
+    [(row, col), ...], each by the definition alone (O(R C) per slot), for images too
+    large for dft2_packed. Slot (row, col) holds, by the layout of dft2_packed:
+      0 < col < C/2 : Re Y[row, col];  C/2 < col : Im Y[row, C - col];
+      col in {0, C/2}: row in {0, R/2} -> Y[row, col]; 0 < row < R/2 -> Re Y[row, col];
+                       R/2 < row -> Im Y[R - row, col].
+    """
+    x = np.asarray(x, dtype=np.float64)
+    R, C = x.shape
+    _check_p(R)
+    _check_p(C)
+    out = []
+    for row, col in slots:
+        if 0 < col < C // 2:
+            k1, k2, part = row, col, "re"
+        elif col > C // 2:
+            k1, k2, part = row, C - col, "im"
+        elif row == 0 or row == R // 2 or row < R // 2:
+            k1, k2, part = row, col, "re"
+        else:
+            k1, k2, part = R - row, col, "im"
+        ar = 2.0 * np.pi * ((k1 * np.arange(R)) % R) / R
+        ac = 2.0 * np.pi * ((k2 * np.arange(C)) % C) / C
+        Y = np.exp(-1j * ar) @ x @ np.exp(-1j * ac)
+        out.append(Y.real if part == "re" else Y.imag)
+    return np.array(out)

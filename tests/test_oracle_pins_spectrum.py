@@ -161,3 +161,31 @@ def test_2d_pins_catch_planted_mistakes(golden):
         if not np.allclose(oracle.unpack2_spectrum(mutant(x)), np.fft.fft2(x), atol=1e-9):
             caught = True
         assert caught, mutant.__name__
+
+
+def test_2d_single_slots_hand_values(golden):
+    for (R, C), xs, ys in golden("packed2d_hand_values.txt"):
+        R, C = int(R), int(C)
+        x = np.array([float(v) for v in xs]).reshape(R, C)
+        y = np.array([float(v) for v in ys]).reshape(R, C)
+        slots = [(r, c) for r in range(R) for c in range(C)]
+        np.testing.assert_allclose(oracle.dft2_packed_at(x, slots), y.ravel(), atol=1e-12)
+
+
+@pytest.mark.parametrize("R,C", [(8, 16), (16, 4), (2, 8)])
+def test_2d_single_slots_read_fft2(R, C):
+    """Each slot is Re or Im of the fft2 entry that the layout assigns it."""
+    x = normal(51, (R, C))
+    F = np.fft.fft2(x)
+    slots = [(r, c) for r in range(R) for c in range(C)]
+    got = oracle.dft2_packed_at(x, slots)
+    for (r, c), v in zip(slots, got):
+        if 0 < c < C // 2:
+            want = F[r, c].real
+        elif c > C // 2:
+            want = F[r, C - c].imag
+        elif r <= R // 2:
+            want = F[r, c].real
+        else:
+            want = F[R - r, c].imag
+        assert abs(v - want) <= 1e-10, (r, c)
