@@ -502,6 +502,34 @@ def run_ours(args):
             del lay, xm, ym
     layer["single_layer_train_step_peak_memory_d4096_bf16"] = memory
 
+    # ---- 2-D rdFFT and the explicit-spectrum cast (beside the step, not in it)
+    spectral = {}
+    for (n2, R2, C2, dt2, name2) in ((8, 4096, 4096, torch.bfloat16, "bf16_8x4096x4096"),
+                                     (64, 1024, 1024, torch.float32, "f32_64x1024x1024")):
+        imgs = torch.randn(n2, R2, C2, device=dev, generator=gen).to(dt2)
+        nbytes = imgs.numel() * imgs.element_size()
+        g2 = graph_of(lambda: (rd.rdfft2_fwd(imgs), rd.rdfft2_inv(imgs)), torch)
+        t2 = time_graph(g2, 10, torch)
+        gf = graph_of(lambda: rd.rdfft2_fwd(imgs), torch)
+        tf = time_graph(gf, 1, torch)                   # one forward (rescales the data once)
+        spectral[f"rdfft2_{name2}"] = {
+            "fwd_inv_ms": round(1e3 * t2, 3), "fwd_ms": round(1e3 * tf, 3),
+            "effective_GBs": round(2 * 2 * nbytes / t2 / 1e9, 1),     # read + write once per transform
+            "moved_GBs": round(2 * 4 * nbytes / t2 / 1e9, 1),         # row half + column half, each r + w
+            "note": "effective = minimum in-place traffic (read + write once) / time; the row and "
+                    "column kernels each read and write the data once"}
+        del imgs, g2, gf
+    rows_c = ELEMS // 512 * 64                      # 128 MiB packed + 128 MiB complex: above L2
+    packed = torch.randn(rows_c, 512, device=dev, generator=gen).to(dt)
+    cplx = torch.empty(rows_c, 257, 2, device=dev, dtype=dt)
+    gc2 = graph_of(lambda: rd.rdfft_to_complex(packed, 512, out=cplx), torch)
+    tc = time_graph(gc2, 20, torch)
+    spectral["to_complex_bf16_p512_GBs"] = round((packed.numel() + cplx.numel()) * 2 / tc / 1e9, 1)
+    gc3 = graph_of(lambda: rd.rdfft_from_complex(cplx, out=packed), torch)
+    tc3 = time_graph(gc3, 20, torch)
+    spectral["from_complex_bf16_p512_GBs"] = round((packed.numel() + cplx.numel()) * 2 / tc3 / 1e9, 1)
+    del packed, cplx, gc2, gc3
+
     # ---- CPU oracle on a bounded sample (rank 0, N = 1 only)
     cpu = None
     if world == 1 and rank == 0:
@@ -526,6 +554,7 @@ def run_ours(args):
         "breakdown": breakdown,
         "single_launch_cold_ms": lat,
         "layer": layer,
+        "spectral": spectral,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "clocks": clocks,
@@ -547,6 +576,8 @@ PROFILE_CASES = {
     "rdfft_bf16_4096_inv": ("rows", (4096, "bf16", "inv")),
     "rdfft_f32_4096_fwd": ("rows", (4096, "f32", "fwd")),
     "rdfft_bf16_4096_inv_config": ("rows_small", (4096, "bf16", "inv")),
+    "rdfft2_bf16_4096_fwd": ("image", (4096, 4096, "bf16", "fwd")),
+    "rdfft2_bf16_4096_inv": ("image", (4096, 4096, "bf16", "inv")),
     "circ_fwd_d4096_p512_b4096": ("circ", (4096, 4096, 512, "fwd")),
     "circ_bwdx_d4096_p512_b4096": ("circ", (4096, 4096, 512, "bwdx")),
     "circ_bwdc_d4096_p512_b4096": ("circ", (4096, 4096, 512, "bwdc")),
@@ -566,7 +597,15 @@ def run_profile_case(name: str) -> int:
     dev = torch.device("cuda", 0)
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
-    if kind in ("rows", "rows_small"):
+    if kind == "image":
+        R, C, dts, d = a
+        dt = torch.bfloat16 if dts == "bf16" else torch.float32
+        x = torch.randn(160 * 1024 * 1024 // (R * C * 2), R, C, device=dev, generator=gen).to(dt)
+        fn, undo = (rd.rdfft2_fwd, rd.rdfft2_inv) if d == "fwd" else (rd.rdfft2_inv, rd.rdfft2_fwd)
+        for _ in range(4):
+            fn(x)
+            undo(x)
+    elif kind in ("rows", "rows_small"):
         p, dts, d = a
         dt = torch.bfloat16 if dts == "bf16" else torch.float32
         esz = 2 if dts == "bf16" else 4

@@ -9,6 +9,9 @@ raises, and the functions accept CUDA tensors only.
 Tensor functions (torch is used for device memory and the current stream):
     rdfft_fwd(t, p)                       in place, packed spectrum of each row
     rdfft_inv(t, p)                       in place, inverse
+    rdfft_to_complex(t, p)                (..., p/2+1, 2) complex bins, out of place
+    rdfft_from_complex(z)                 packed rows from complex bins, out of place
+    rdfft2_fwd(t) / rdfft2_inv(t)         in place, 2-D packed spectrum of (..., R, C)
     circ_fwd(x, c_hat, p, y=None)         y = W x
     circ_bwd(g, x, c_hat, p, grad_x=..., grad_c=...)
     circ_prepare(c)                       c_hat = packed rdfft_fwd of fp32 c
@@ -18,7 +21,8 @@ Raw entry points on integer device pointers: ``lib`` (the ctypes handle).
 from __future__ import annotations
 
 _EXPORTS = ("RDFFT_BF16", "RDFFT_F32", "RDFFT_ETIMEOUT", "RdfftError", "circ_bwd", "circ_fwd", "circ_prepare",
-            "lib", "lib_path", "rdfft_fwd", "rdfft_inv", "take_device_error", "selftest_wait_timeout")
+            "lib", "lib_path", "rdfft_fwd", "rdfft_inv", "rdfft_to_complex", "rdfft_from_complex", "rdfft2_fwd",
+            "rdfft2_inv", "take_device_error", "selftest_wait_timeout")
 _LAYER = ("BlockCirculantLinear", "block_circulant")
 
 __all__ = list(_EXPORTS + _LAYER)

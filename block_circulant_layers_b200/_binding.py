@@ -22,9 +22,14 @@ lib = ctypes.CDLL(lib_path)
 _i64, _int, _vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
 lib.rdfft_fwd.argtypes = [_vp, _i64, _int, _int, _vp]
 lib.rdfft_inv.argtypes = [_vp, _i64, _int, _int, _vp]
+lib.rdfft_to_complex.argtypes = [_vp, _vp, _i64, _int, _int, _vp]
+lib.rdfft_from_complex.argtypes = [_vp, _vp, _i64, _int, _int, _vp]
+lib.rdfft2_fwd.argtypes = [_vp, _i64, _int, _int, _int, _vp]
+lib.rdfft2_inv.argtypes = [_vp, _i64, _int, _int, _int, _vp]
 lib.circ_fwd.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _vp]
-for _f in (lib.rdfft_fwd, lib.rdfft_inv, lib.circ_fwd, lib.circ_bwd):
+for _f in (lib.rdfft_fwd, lib.rdfft_inv, lib.rdfft_to_complex, lib.rdfft_from_complex, lib.rdfft2_fwd,
+           lib.rdfft2_inv, lib.circ_fwd, lib.circ_bwd):
     _f.restype = _int
 lib.rdfft_strerror.argtypes = [_int]
 lib.rdfft_strerror.restype = ctypes.c_char_p
@@ -85,6 +90,69 @@ def rdfft_inv(t: torch.Tensor, p: int) -> torch.Tensor:
         raise ValueError("numel must be a multiple of p")
     with torch.cuda.device(t.device):
         _check(lib.rdfft_inv(t.data_ptr(), t.numel() // p, p, _dtype_code(t), _stream(t)), "rdfft_inv")
+    return t
+
+
+def rdfft_to_complex(t: torch.Tensor, p: int, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Complex bins Y_0..Y_{p/2} of packed rows `t` (..., p), out of place, as a tensor of
+    shape (..., p/2 + 1, 2) of t's dtype holding (re, im); for float32 use
+    torch.view_as_complex on it."""
+    _cuda_dense(t, "t")
+    if p <= 0 or t.shape[-1] != p:
+        raise ValueError("the last dimension of t must be p")
+    shape = t.shape[:-1] + (p // 2 + 1, 2)
+    if out is None:
+        out = torch.empty(shape, dtype=t.dtype, device=t.device)
+    _cuda_dense(out, "out")
+    if out.shape != shape or out.dtype != t.dtype:
+        raise ValueError(f"out must have shape {tuple(shape)} and dtype {t.dtype}")
+    with torch.cuda.device(t.device):
+        _check(lib.rdfft_to_complex(t.data_ptr(), out.data_ptr(), t.numel() // p, p, _dtype_code(t), _stream(t)),
+               "rdfft_to_complex")
+    return out
+
+
+def rdfft_from_complex(z: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
+    """Packed rows (..., p) from complex bins z (..., p/2 + 1, 2), out of place."""
+    _cuda_dense(z, "z")
+    if z.dim() < 2 or z.shape[-1] != 2:
+        raise ValueError("z must have shape (..., p/2 + 1, 2)")
+    p = 2 * (z.shape[-2] - 1)
+    shape = z.shape[:-2] + (p,)
+    if out is None:
+        out = torch.empty(shape, dtype=z.dtype, device=z.device)
+    _cuda_dense(out, "out")
+    if out.shape != shape or out.dtype != z.dtype:
+        raise ValueError(f"out must have shape {tuple(shape)} and dtype {z.dtype}")
+    rows = out.numel() // p if p > 0 else 0
+    with torch.cuda.device(z.device):
+        _check(lib.rdfft_from_complex(z.data_ptr(), out.data_ptr(), rows, p, _dtype_code(z), _stream(z)),
+               "rdfft_from_complex")
+    return out
+
+
+def _images(t: torch.Tensor):
+    if t.dim() < 2:
+        raise ValueError("t must have shape (..., R, C)")
+    R, C = t.shape[-2], t.shape[-1]
+    return t.numel() // (R * C) if R * C else 0, R, C
+
+
+def rdfft2_fwd(t: torch.Tensor) -> torch.Tensor:
+    """In-place 2-D rdFFT of every R x C image in the last two dimensions of `t`."""
+    _cuda_dense(t, "t")
+    n, R, C = _images(t)
+    with torch.cuda.device(t.device):
+        _check(lib.rdfft2_fwd(t.data_ptr(), n, R, C, _dtype_code(t), _stream(t)), "rdfft2_fwd")
+    return t
+
+
+def rdfft2_inv(t: torch.Tensor) -> torch.Tensor:
+    """In-place inverse 2-D rdFFT (with 1/(R C)) of every packed R x C spectrum in `t`."""
+    _cuda_dense(t, "t")
+    n, R, C = _images(t)
+    with torch.cuda.device(t.device):
+        _check(lib.rdfft2_inv(t.data_ptr(), n, R, C, _dtype_code(t), _stream(t)), "rdfft2_inv")
     return t
 
 

@@ -9,6 +9,7 @@
 
 #include <vector>
 
+#include "rdfft2d_steps.cuh"
 #include "rdfft_steps.cuh"
 
 namespace rdfft {
@@ -44,6 +45,14 @@ void emu_hartley_rest(float* tile, int nr, T* rows) {
     else merged_orbit<G, K, false, 0, 0, T>(tile, r, mu % NB, (T*)nullptr, false);
   }
   if constexpr (!LAST) emu_hartley_rest<G, K + 1, T>(tile, nr, rows);
+}
+
+template <class G, int W, int NT, int K>
+void emu_col_passes(float* tile) {
+  if constexpr (K < G::NPASS) {
+    for (int tid = 0; tid < NT; ++tid) cols_orbit_pass<G, K>(tile, W, tid, NT);
+    emu_col_passes<G, W, NT, K + 1>(tile);
+  }
 }
 
 // Emulates the row transform of geometry G with ROWS rows per CTA.
@@ -105,6 +114,58 @@ void emu_hartley_inverse(T* data, int64_t rows) {
   }
 }
 
+// Column half of the 2-D transform, CTA by CTA as k_cols / k_cols_small run it.
+template <int R, bool INV, typename T>
+void emu_cols(T* data, int64_t images, int C) {
+  if constexpr (R <= 32) {
+    for (int64_t img = 0; img < images; ++img)
+      for (int k = 0; k <= C / 2; ++k) col_small<R, INV, T>(data + img * (int64_t)R * C, C, k);
+  } else {
+    using CT = ColTiling<R>;
+    constexpr int W = CT::W, NT = CT::NT;
+    using G = ColGeo<R, W>;
+    constexpr int TPR = G::TPR;
+    std::vector<float> tile(G::words(W), 0.0f);
+    std::vector<float> regs((size_t)W * TPR * G::E);
+    const int ngroups = col_groups(C, W / 2);
+    for (int64_t img = 0; img < images; ++img) {
+      T* base = data + img * (int64_t)R * C;
+      for (int grp = 0; grp < ngroups; ++grp) {
+        const int k0 = grp * (W / 2);
+        float* t = tile.data();
+        for (int tid = 0; tid < NT; ++tid) cols_load<G, W, T>(t, base, C, k0, tid, NT);
+        if (INV)
+          for (int tid = 0; tid < NT; ++tid) cols_unpair_mirror<G, W>(t, C, k0, tid, NT);
+        for (int i = 0; i < W * TPR; ++i) {
+          float(&a)[G::E] = *reinterpret_cast<float(*)[G::E]>(&regs[(size_t)i * G::E]);
+          fwd_pass0_load_tile<G>(a, i % TPR, t + G::row_base(i / TPR));
+        }
+        for (int i = 0; i < W * TPR; ++i) {
+          float(&a)[G::E] = *reinterpret_cast<float(*)[G::E]>(&regs[(size_t)i * G::E]);
+          fwd_pass0_finish<G>(a, i % TPR, t + G::row_base(i / TPR));
+        }
+        emu_col_passes<G, W, NT, 1>(t);
+        for (int tid = 0; tid < NT; ++tid) {
+          if (INV) cols_store_inv<G, W, T>(t, base, C, k0, tid, NT);
+          else cols_store_fwd<G, W, T>(t, base, C, k0, tid, NT);
+        }
+      }
+    }
+  }
+}
+
+template <bool INV, typename T>
+int emu_cols_t(T* data, int64_t images, int R, int C) {
+#define RD_CCASE(RR) \
+  case RR: emu_cols<RR, INV, T>(data, images, C); return 0;
+  switch (R) {
+    RD_CCASE(2) RD_CCASE(4) RD_CCASE(8) RD_CCASE(16) RD_CCASE(32) RD_CCASE(64) RD_CCASE(128)
+    RD_CCASE(256) RD_CCASE(512) RD_CCASE(1024) RD_CCASE(2048) RD_CCASE(4096)
+    default: return 1;
+  }
+#undef RD_CCASE
+}
+
 template <typename T>
 int emu_t(void* data, int64_t rows, int p, bool inv, int ept) {
   T* d = static_cast<T*>(data);
@@ -152,6 +213,28 @@ int rdfft_emulate_hartley_inverse(void* data, int64_t rows, int p, int dtype) {
 int rdfft_emulate_layer_rows(void* data, int64_t rows, int p, int dtype, int inverse) {
   if (dtype == 0) return rdfft::emu_t<float>(data, rows, p, inverse != 0, 32);
   return rdfft::emu_t<rdfft::bf16_t>(data, rows, p, inverse != 0, 32);
+}
+
+// Emulated rdfft2_fwd / rdfft2_inv on host images (row kernel, then column kernel,
+// or the reverse); returns 1 for an unsupported R or C.
+int rdfft2_emulate(void* data, int64_t images, int R, int C, int dtype, int inverse) {
+  const int64_t rows = images * R;
+  if (dtype == 0) {
+    float* d = static_cast<float*>(data);
+    if (!inverse) {
+      if (rdfft::emu_t<float>(d, rows, C, false, 0)) return 1;
+      return rdfft::emu_cols_t<false>(d, images, R, C);
+    }
+    if (rdfft::emu_cols_t<true>(d, images, R, C)) return 1;
+    return rdfft::emu_t<float>(d, rows, C, true, 0);
+  }
+  rdfft::bf16_t* d = static_cast<rdfft::bf16_t*>(data);
+  if (!inverse) {
+    if (rdfft::emu_t<rdfft::bf16_t>(d, rows, C, false, 0)) return 1;
+    return rdfft::emu_cols_t<false>(d, images, R, C);
+  }
+  if (rdfft::emu_cols_t<true>(d, images, R, C)) return 1;
+  return rdfft::emu_t<rdfft::bf16_t>(d, rows, C, true, 0);
 }
 
 // Positions of the first n elements of the generic orbit with residue r of a pass

@@ -16,6 +16,14 @@ cudaError_t take_rows_device_error(unsigned int* flags);
 // Launches a kernel whose bounded wait must time out (self-test of the error path).
 cudaError_t launch_wait_selftest(cudaStream_t s);
 
+// Packed <-> rFFT complex layout conversion (see rdfft_to_complex / rdfft_from_complex).
+cudaError_t launch_convert(const void* in, void* out, int64_t rows, int p, int dtype, bool to_complex,
+                           cudaStream_t s);
+
+// Column half of the 2-D rdFFT of `images` images of R x C (see rdfft2_fwd / rdfft2_inv):
+// forward column transform with the pair combine, or its inverse.
+cudaError_t launch_cols(void* data, int64_t images, int R, int C, int dtype, bool inverse, cudaStream_t s);
+
 // Block-circulant layer forward: y = W x (see circ_fwd in rdfft.h).
 cudaError_t launch_circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p,
                             int dtype, cudaStream_t s);

@@ -44,6 +44,41 @@ bool overlap(const void* a, size_t na, const void* b, size_t nb) {
   return x < y + nb && y < x + na;
 }
 
+int convert_call(const void* in, void* out, int64_t rows, int p, int dtype, bool to_complex,
+                 rdfft_stream_t stream) {
+  if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
+  if (!pow2_in_range(p) || rows < 0) return RDFFT_EINVAL;
+  if (rows == 0) return RDFFT_OK;
+  if (in == nullptr || out == nullptr) return RDFFT_ENULL;
+  if (!aligned16(in) || !aligned16(out)) return RDFFT_EALIGN;
+  const size_t es = dtype == RDFFT_F32 ? 4 : 2;
+  const size_t packed_bytes = (size_t)rows * p * es, cplx_bytes = (size_t)rows * (p + 2) * es;
+  if (overlap(in, to_complex ? packed_bytes : cplx_bytes, out, to_complex ? cplx_bytes : packed_bytes))
+    return RDFFT_EOVERLAP;
+  return finish(rdfft::launch_convert(in, out, rows, p, dtype, to_complex, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+// The 2-D transform: rows then columns (forward), columns then rows (inverse), in
+// place; both halves are enqueued on the same stream.
+int image_call(void* data, int64_t images, int R, int C, int dtype, rdfft_stream_t stream, bool inverse) {
+  if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
+  if (!pow2_in_range(R) || !pow2_in_range(C) || images < 0) return RDFFT_EINVAL;
+  if (images > INT64_MAX / ((int64_t)R * C)) return RDFFT_EINVAL;
+  if (images == 0) return RDFFT_OK;
+  if (data == nullptr) return RDFFT_ENULL;
+  if (!aligned16(data)) return RDFFT_EALIGN;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t rows = images * R;
+  if (!inverse) {
+    const cudaError_t e = rdfft::launch_rows(data, rows, C, dtype, false, s);
+    if (e != cudaSuccess) return finish(e);
+    return finish(rdfft::launch_cols(data, images, R, C, dtype, false, s));
+  }
+  const cudaError_t e = rdfft::launch_cols(data, images, R, C, dtype, true, s);
+  if (e != cudaSuccess) return finish(e);
+  return finish(rdfft::launch_rows(data, rows, C, dtype, true, s));
+}
+
 }  // namespace
 
 extern "C" {
@@ -54,6 +89,22 @@ int rdfft_fwd(void* data, int64_t rows, int p, int dtype, rdfft_stream_t stream)
 
 int rdfft_inv(void* data, int64_t rows, int p, int dtype, rdfft_stream_t stream) {
   return rows_call(data, rows, p, dtype, stream, true);
+}
+
+int rdfft_to_complex(const void* packed, void* cplx, int64_t rows, int p, int dtype, rdfft_stream_t stream) {
+  return convert_call(packed, cplx, rows, p, dtype, true, stream);
+}
+
+int rdfft_from_complex(const void* cplx, void* packed, int64_t rows, int p, int dtype, rdfft_stream_t stream) {
+  return convert_call(cplx, packed, rows, p, dtype, false, stream);
+}
+
+int rdfft2_fwd(void* data, int64_t images, int R, int C, int dtype, rdfft_stream_t stream) {
+  return image_call(data, images, R, C, dtype, stream, false);
+}
+
+int rdfft2_inv(void* data, int64_t images, int R, int C, int dtype, rdfft_stream_t stream) {
+  return image_call(data, images, R, C, dtype, stream, true);
 }
 
 int circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p, int dtype,
@@ -123,6 +174,6 @@ int rdfft_selftest_wait_timeout(rdfft_stream_t stream) {
   return finish(rdfft::launch_wait_selftest(reinterpret_cast<cudaStream_t>(stream)));
 }
 
-int rdfft_version(void) { return 100; }
+int rdfft_version(void) { return 110; }
 
 }  // extern "C"

@@ -6,10 +6,12 @@
  * Source of the method: "Memory-Efficient Training with In-Place FFT
  * Implementation" (arXiv 2511.01385). Citations below name the web page that
  * describes a step and its section:
- *   [summary]     the AI-written summary page, sections "Approach" and "Problem";
+ *   [summary]     the AI-written summary page, sections "Approach", "Problem" and
+ *                 "Limitations";
  *   [notes]       the paper-notes page, method section, items "Squeeze N+2 -> N",
  *                 "Proposition 1", "In-place IFFT design" and "Circulant matrix
- *                 training adaptation", and its "Training strategy" list.
+ *                 training adaptation", its "Training strategy" list and its
+ *                 "Limitations and outlook".
  *
  * Packed layout of a row of length p (every transform buffer uses it)
  * ([summary] Approach; [notes] "Squeeze N+2 -> N"): the spectrum Y of a real row
@@ -34,7 +36,8 @@
  *   - Return value: RDFFT_OK, or an error code. Argument errors are reported before
  *     anything is enqueued. RDFFT_ECUDA means a CUDA call failed when enqueuing;
  *     rdfft_strerror() then includes the CUDA message, which is kept per host
- *     thread. Empty work (rows == 0 or B == 0) returns RDFFT_OK and enqueues nothing.
+ *     thread. Empty work (rows == 0, images == 0 or B == 0) returns RDFFT_OK and
+ *     enqueues nothing.
  */
 #ifndef RDFFT_H
 #define RDFFT_H
@@ -87,6 +90,53 @@ int rdfft_fwd(void* data, int64_t rows, int p, int dtype, rdfft_stream_t stream)
  *   data  : rows x p packed spectra of `dtype`, overwritten by the real rows.
  */
 int rdfft_inv(void* data, int64_t rows, int p, int dtype, rdfft_stream_t stream);
+
+/*
+ * rdfft_to_complex -- explicit complex bins of packed rows, out of place.
+ * [summary] "Limitations": the packed layout encodes the spectrum implicitly, and
+ * reaching the complex values (for spectral filtering, say) takes a cast that cannot
+ * stay in the same buffer, since p reals become p/2 + 1 complex values. This is that
+ * cast; it only moves values (bf16 stays bf16, bit for bit).
+ *   packed : rows x p of `dtype` in the packed layout above, read only.
+ *   cplx   : rows x (p/2 + 1) interleaved (re, im) pairs of `dtype` (rows x (p + 2)
+ *            elements), written: bin k = (slot k, slot p-k) for 0 < k < p/2, bins 0
+ *            and p/2 = (slot 0 or p/2, 0). Must not overlap `packed` (RDFFT_EOVERLAP).
+ *   rows >= 0; p a power of two in [2, 4096].
+ */
+int rdfft_to_complex(const void* packed, void* cplx, int64_t rows, int p, int dtype, rdfft_stream_t stream);
+
+/*
+ * rdfft_from_complex -- packed rows from complex bins, out of place (the reverse cast
+ * of rdfft_to_complex). The imaginary parts of bins 0 and p/2 are not read: they are
+ * zero for the spectrum of a real row, and the packed layout has no slot for them.
+ *   cplx   : rows x (p/2 + 1) interleaved (re, im) pairs of `dtype`, read only.
+ *   packed : rows x p of `dtype`, written. Must not overlap `cplx` (RDFFT_EOVERLAP).
+ */
+int rdfft_from_complex(const void* cplx, void* packed, int64_t rows, int p, int dtype, rdfft_stream_t stream);
+
+/*
+ * rdfft2_fwd -- 2-D rdFFT of `images` real images of R x C (row-major), in place.
+ * [notes] "Limitations and outlook" leaves the 2-D transform open; this library takes
+ * the packed layout per axis, so that every slot of the image holds one real number
+ * of its 2-D spectrum Y[k1, k2] = sum_{r,c} x[r,c] exp(-2 pi i (k1 r/R + k2 c/C)):
+ *   columns 0 < k2 < C/2 : slot [k1][k2] = Re Y[k1, k2], slot [k1][C-k2] = Im Y[k1, k2]
+ *                          for every k1 < R;
+ *   columns k2 = 0, C/2  : Y[., k2] is conjugate symmetric in k1 and is stored down
+ *                          the column in the 1-D packed layout above.
+ * Computed as rdfft_fwd of the R rows of each image, then an in-place column
+ * transform that combines the columns k2 and C - k2 (two kernels, each reading and
+ * writing the data once).
+ *   data   : images x R x C of `dtype`, overwritten by the packed 2-D spectra.
+ *   images >= 0; R, C powers of two in [2, 4096].
+ */
+int rdfft2_fwd(void* data, int64_t images, int R, int C, int dtype, rdfft_stream_t stream);
+
+/*
+ * rdfft2_inv -- inverse of rdfft2_fwd (with the 1/(R C) of the inverse DFT), in place:
+ * the column inverse (in its Hartley form, (1/R) M rdFFT M with M the mirror of a
+ * packed row) and then rdfft_inv of the rows.
+ */
+int rdfft2_inv(void* data, int64_t images, int R, int C, int dtype, rdfft_stream_t stream);
 
 /*
  * circ_fwd -- block-circulant linear layer, forward.

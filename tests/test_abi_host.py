@@ -25,6 +25,10 @@ def lib():
     i64, i, vp = ctypes.c_int64, ctypes.c_int, ctypes.c_void_p
     L.rdfft_fwd.argtypes = [vp, i64, i, i, vp]
     L.rdfft_inv.argtypes = [vp, i64, i, i, vp]
+    L.rdfft_to_complex.argtypes = [vp, vp, i64, i, i, vp]
+    L.rdfft_from_complex.argtypes = [vp, vp, i64, i, i, vp]
+    L.rdfft2_fwd.argtypes = [vp, i64, i, i, i, vp]
+    L.rdfft2_inv.argtypes = [vp, i64, i, i, i, vp]
     L.circ_fwd.argtypes = [vp, vp, vp, i64, i, i, i, vp]
     L.circ_bwd.argtypes = [vp, vp, vp, vp, vp, i64, i, i, i, vp]
     L.rdfft_strerror.argtypes = [i]
@@ -40,8 +44,9 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for n in ("rdfft_fwd", "rdfft_inv", "circ_fwd", "circ_bwd", "rdfft_strerror", "rdfft_version",
-              "rdfft_take_device_error", "rdfft_selftest_wait_timeout"):
+    for n in ("rdfft_fwd", "rdfft_inv", "rdfft_to_complex", "rdfft_from_complex", "rdfft2_fwd", "rdfft2_inv",
+              "circ_fwd", "circ_bwd", "rdfft_strerror", "rdfft_version", "rdfft_take_device_error",
+              "rdfft_selftest_wait_timeout"):
         assert n in names
 
 
@@ -76,6 +81,36 @@ def test_rdfft_argument_errors(lib):
         assert fn(A, -1, 512, F32, None) == EINVAL
         assert fn(A, 4, 512, 2, None) == EDTYPE
         assert fn(A + 4, 4, 512, BF16, None) == EALIGN
+
+
+def test_complex_cast_argument_errors(lib):
+    for fn in (lib.rdfft_to_complex, lib.rdfft_from_complex):
+        assert fn(None, None, 0, 512, F32, None) == OK
+        assert fn(None, Bp, 4, 512, F32, None) == ENULL
+        assert fn(A, None, 4, 512, F32, None) == ENULL
+        assert fn(A, Bp, 4, 6, F32, None) == EINVAL
+        assert fn(A, Bp, -2, 512, F32, None) == EINVAL
+        assert fn(A, Bp, 4, 512, 3, None) == EDTYPE
+        assert fn(A + 8, Bp, 4, 512, F32, None) == EALIGN
+        assert fn(A, Bp + 2, 4, 512, BF16, None) == EALIGN
+        assert fn(A, A, 4, 512, F32, None) == EOVERLAP
+    # packed rows 4 x 512 f32 = 8192 B; complex rows 4 x 514 f32 = 8224 B (only
+    # overlapping pairs here: a disjoint pair would pass validation and launch)
+    assert lib.rdfft_to_complex(A, A + 8176, 4, 512, F32, None) == EOVERLAP
+    assert lib.rdfft_from_complex(A, A + 8208, 4, 512, F32, None) == EOVERLAP
+
+
+def test_2d_argument_errors(lib):
+    for fn in (lib.rdfft2_fwd, lib.rdfft2_inv):
+        assert fn(None, 0, 64, 64, F32, None) == OK
+        assert fn(None, 2, 64, 64, F32, None) == ENULL
+        assert fn(A, 2, 48, 64, F32, None) == EINVAL
+        assert fn(A, 2, 64, 8192, F32, None) == EINVAL
+        assert fn(A, 2, 1, 64, F32, None) == EINVAL
+        assert fn(A, -1, 64, 64, F32, None) == EINVAL
+        assert fn(A, 1 << 40, 4096, 4096, F32, None) == EINVAL      # images * R * C overflows int64
+        assert fn(A, 2, 64, 64, 7, None) == EDTYPE
+        assert fn(A + 2, 2, 64, 64, BF16, None) == EALIGN
 
 
 def test_circ_argument_errors(lib):
