@@ -133,9 +133,10 @@ void emu_cols(T* data, int64_t images, int C) {
       for (int grp = 0; grp < ngroups; ++grp) {
         const int k0 = grp * (W / 2);
         float* t = tile.data();
-        for (int tid = 0; tid < NT; ++tid) cols_load<G, W, T>(t, base, C, k0, tid, NT);
-        if (INV)
-          for (int tid = 0; tid < NT; ++tid) cols_unpair_mirror<G, W>(t, C, k0, tid, NT);
+        for (int tid = 0; tid < NT; ++tid) {
+          if (INV) cols_load_unpair<G, W, NT, T>(t, base, C, k0, tid);
+          else cols_load<G, W, NT, T>(t, base, C, k0, tid);
+        }
         for (int i = 0; i < W * TPR; ++i) {
           float(&a)[G::E] = *reinterpret_cast<float(*)[G::E]>(&regs[(size_t)i * G::E]);
           fwd_pass0_load_tile<G>(a, i % TPR, t + G::row_base(i / TPR));
@@ -146,8 +147,8 @@ void emu_cols(T* data, int64_t images, int C) {
         }
         emu_col_passes<G, W, NT, 1>(t);
         for (int tid = 0; tid < NT; ++tid) {
-          if (INV) cols_store_inv<G, W, T>(t, base, C, k0, tid, NT);
-          else cols_store_fwd<G, W, T>(t, base, C, k0, tid, NT);
+          if (INV) cols_store_inv<G, W, NT, T>(t, base, C, k0, tid);
+          else cols_store_fwd<G, W, NT, T>(t, base, C, k0, tid);
         }
       }
     }
@@ -184,6 +185,18 @@ int emu_t(void* data, int64_t rows, int p, bool inv, int ept) {
 
 }  // namespace
 }  // namespace rdfft
+
+template <class SM, int P>
+static void plan_of(int64_t* out) {
+  out[0] = SM::ROWS;
+  out[1] = SM::RAW_ROW;
+  out[2] = SM::TILE_OFF;
+  out[3] = SM::MBAR_OFF;
+  out[4] = SM::BYTES;
+  out[5] = rdfft::RowGeo<P>::words(SM::ROWS);
+  out[6] = SM::TPR;
+  for (int r = 0; r < SM::ROWS; ++r) out[7 + r] = SM::raw_off(r);
+}
 
 extern "C" {
 
@@ -235,6 +248,23 @@ int rdfft2_emulate(void* data, int64_t images, int R, int C, int dtype, int inve
   }
   if (rdfft::emu_cols_t<true>(d, images, R, C)) return 1;
   return rdfft::emu_t<rdfft::bf16_t>(d, rows, C, true, 0);
+}
+
+// Shared-memory plan of the rows kernel for row length p >= 64 and dtype: out[0..6] =
+// rows per CTA, bytes per staged row, tile offset, mbarrier offset, total bytes, tile
+// words, threads per row; out[7 + r] = byte offset of staged row r (out must hold
+// 7 + rows per CTA values). Returns 1 for an unsupported p.
+int rdfft_row_smem_plan(int p, int dtype, int64_t* out) {
+#define RD_PCASE(PP)                                                                   \
+  case PP:                                                                             \
+    if (dtype == 0) plan_of<rdfft::RowSmem<PP, float>, PP>(out);                       \
+    else plan_of<rdfft::RowSmem<PP, rdfft::bf16_t>, PP>(out);                          \
+    return 0;
+  switch (p) {
+    RD_PCASE(64) RD_PCASE(128) RD_PCASE(256) RD_PCASE(512) RD_PCASE(1024) RD_PCASE(2048) RD_PCASE(4096)
+    default: return 1;
+  }
+#undef RD_PCASE
 }
 
 // Positions of the first n elements of the generic orbit with residue r of a pass

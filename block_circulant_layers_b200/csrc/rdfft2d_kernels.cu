@@ -34,12 +34,9 @@ k_cols(T* __restrict__ data, int C, int ngroups) {
   T* base = data + img * (int64_t)R * C;
   const int tid = threadIdx.x;
 
-  cols_load<G, W, T>(tile, base, C, k0, tid, NT);
+  if constexpr (INV) cols_load_unpair<G, W, NT, T>(tile, base, C, k0, tid);
+  else cols_load<G, W, NT, T>(tile, base, C, k0, tid);
   __syncthreads();
-  if constexpr (INV) {
-    cols_unpair_mirror<G, W>(tile, C, k0, tid, NT);
-    __syncthreads();
-  }
   // pass 0 in place in the tile: every row of a round gathers, barrier, scatters
   const int v = tid % TPR;
   for (int r0 = 0; r0 < W; r0 += NT / TPR) {
@@ -51,8 +48,8 @@ k_cols(T* __restrict__ data, int C, int ngroups) {
   }
   run_col_passes<G, W, NT, 1>(tile, tid);
   __syncthreads();
-  if constexpr (INV) cols_store_inv<G, W, T>(tile, base, C, k0, tid, NT);
-  else cols_store_fwd<G, W, T>(tile, base, C, k0, tid, NT);
+  if constexpr (INV) cols_store_inv<G, W, NT, T>(tile, base, C, k0, tid);
+  else cols_store_fwd<G, W, NT, T>(tile, base, C, k0, tid);
 }
 
 // Columns of R <= 32: one thread per (image, left column k <= C/2).

@@ -31,12 +31,13 @@
 namespace rdfft {
 
 // Columns per CTA and CTA size for column length R >= 64: the tile (W columns of R
-// fp32 plus pad) stays near 64 KiB for R <= 1024 and 132 KiB above.
+// fp32 plus pad) stays near 64 KiB for R <= 1024 and 132 KiB above; one thread per
+// TPR-th of every column (up to 1024 threads), at least 128.
 template <int R>
 struct ColTiling {
   static constexpr int W = R >= 4096 ? 8 : (R >= 1024 ? 16 : 32);
   static constexpr int TPR = Geo<R, kEPT>::TPR;
-  static constexpr int NT = W * TPR > 512 ? 512 : (W * TPR < 128 ? 128 : W * TPR);
+  static constexpr int NT = W * TPR > 1024 ? 1024 : (W * TPR < 128 ? 128 : W * TPR);
 };
 
 // The row geometry of a column tile. For R >= 1024 (a warp per tile row in the
@@ -67,43 +68,88 @@ RD_HD int strip_col(int j, int H, int k0, int C) {
 // Number of strip pairs (CTAs) per image: left columns 0..C/2.
 RD_HD constexpr int col_groups(int C, int H) { return (C / 2 + H) / H; }
 
-// HBM -> tile: element (r, column of tile row j) to tile row j, position r.
-template <class G, int W, typename T>
-RD_HD void cols_load(float* tile, const T* img, int C, int k0, int tid, int NT) {
-  constexpr int R = G::P, H = W / 2;
-  for (int idx = tid; idx < R * W; idx += NT) {
-    const int r = idx / W, j = idx % W;
-    const int col = strip_col(j, H, k0, C);
-    tile[G::row_base(j) + G::at(r)] = col >= 0 ? ld(img + (int64_t)r * C + col) : 0.0f;
+// HBM -> tile (forward). Thread tid owns tile row j = tid % W, a fixed image column,
+// and image rows r0 + i STEP (r0 = tid / W, STEP = NT / W), so its tile addresses
+// are one base plus compile-time offsets (STEP and 2^S divide one another) and its
+// global addresses one base plus multiples of STEP rows. Loads are issued in batches
+// of LB before their shared-memory stores, to keep LB loads in flight per thread.
+template <class G, int W, int NT, typename T>
+RD_HD void cols_load(float* tile, const T* img, int C, int k0, int tid) {
+  constexpr int R = G::P, H = W / 2, STEP = NT / W, ITER = R / STEP;
+  constexpr int LB = ITER < 16 ? ITER : 16;
+  static_assert(NT % W == 0 && R % STEP == 0 && ITER % LB == 0, "whole rounds");
+  static_assert(STEP % (1 << G::S) == 0 || (1 << G::S) % STEP == 0, "compile-time tile offsets");
+  const int j = tid % W, r0 = tid / W;
+  const int col = strip_col(j, H, k0, C);
+  float* trow = tile + G::row_base(j) + G::at(r0);
+  const T* src = img + (int64_t)r0 * C + (col >= 0 ? col : 0);
+  const int64_t gstep = (int64_t)STEP * C;
+#pragma unroll
+  for (int i0 = 0; i0 < ITER; i0 += LB) {
+    float v[LB];
+#pragma unroll
+    for (int b = 0; b < LB; ++b) v[b] = col >= 0 ? ld(src + (i0 + b) * gstep) : 0.0f;
+#pragma unroll
+    for (int b = 0; b < LB; ++b) {
+      const int c = (i0 + b) * STEP;
+      trow[c + (c >> G::S)] = v[b];
+    }
   }
 }
 
-// Inverse, first sweep: un-combine each pair (k, C-k) back to the packed column
-// spectra A, B and apply the mirror M to every column (slots 0 and R/2 unchanged).
-// With u, u2 = Re Y at k1, R-k1 and w, w2 = Im Y there:
+// HBM -> tile (inverse), fused with the first sweep of the inverse: un-combine each
+// pair (k, C-k) back to the packed column spectra A, B and apply the mirror M to every
+// column (slots 0 and R/2 unchanged). With u, u2 = Re Y at k1, R-k1 and w, w2 = Im Y:
 //   Ar = (u + u2)/2, Bi = (u2 - u)/2, Br = (w + w2)/2, Ai = (w - w2)/2, and
 //   M A: [k1] = Ar - Ai, [R-k1] = Ar + Ai;  M B: [k1] = Br - Bi, [R-k1] = Br + Bi.
-template <class G, int W>
-RD_HD void cols_unpair_mirror(float* tile, int C, int k0, int tid, int NT) {
-  constexpr int R = G::P, H = W / 2, Q = R / 2;
-  for (int idx = tid; idx < H * Q; idx += NT) {
-    const int jl = idx / Q, k1 = idx % Q;
-    const int k = k0 + jl;
-    if (k1 == 0 || k > C / 2) continue;
-    float* A = tile + G::row_base(jl);
-    const int lo = G::at(k1), hi = G::at(R - k1);
-    if (k > 0 && k < C / 2) {
-      float* B = tile + G::row_base(jl + H);
-      const float u = A[lo], u2 = A[hi], w = B[lo], w2 = B[hi];
-      const float su = u + u2, du = u - u2, sw = w + w2, dw = w - w2;
-      A[lo] = 0.5f * (su - dw);
-      A[hi] = 0.5f * (su + dw);
-      B[lo] = 0.5f * (sw + du);
-      B[hi] = 0.5f * (sw - du);
-    } else {
-      const float a = A[lo], b = A[hi];
-      A[lo] = a - b;
-      A[hi] = a + b;
+// Thread tid owns left column k = k0 + tid % H (and its mirror) and the row pairs
+// (k1, R - k1) for k1 = q0 + i STEP (q0 = tid / H, STEP = NT / H); k1 = 0 stands for
+// the rows (0, R/2), which are copied.
+template <class G, int W, int NT, typename T>
+RD_HD void cols_load_unpair(float* tile, const T* img, int C, int k0, int tid) {
+  constexpr int R = G::P, H = W / 2, Q = R / 2, STEP = NT / H, ITER = Q / STEP;
+  constexpr int LB = ITER < 8 ? ITER : 8;
+  static_assert(NT % H == 0 && Q % STEP == 0 && ITER % LB == 0, "whole rounds");
+  const int jl = tid % H, q0 = tid / H;
+  const int k = k0 + jl;
+  const bool valid = k <= C / 2, paired = k > 0 && k < C / 2;
+  float* A = tile + G::row_base(jl);
+  float* B = tile + G::row_base(jl + H);
+  const T* ca = img + (valid ? k : 0);
+  const T* cb = img + (paired ? C - k : 0);
+#pragma unroll
+  for (int i0 = 0; i0 < ITER; i0 += LB) {
+    float u[LB], u2[LB], w[LB], w2[LB];
+#pragma unroll
+    for (int b = 0; b < LB; ++b) {
+      const int k1 = q0 + (i0 + b) * STEP;
+      const int lo = k1, hi = k1 == 0 ? Q : R - k1;
+      u[b] = valid ? ld(ca + (int64_t)lo * C) : 0.0f;
+      u2[b] = valid ? ld(ca + (int64_t)hi * C) : 0.0f;
+      w[b] = paired ? ld(cb + (int64_t)lo * C) : 0.0f;
+      w2[b] = paired ? ld(cb + (int64_t)hi * C) : 0.0f;
+    }
+#pragma unroll
+    for (int b = 0; b < LB; ++b) {
+      const int k1 = q0 + (i0 + b) * STEP;
+      const int lo = G::at(k1), hi = G::at(k1 == 0 ? Q : R - k1);
+      if (k1 == 0) {
+        A[lo] = u[b];
+        A[hi] = u2[b];
+        B[lo] = w[b];
+        B[hi] = w2[b];
+      } else if (paired) {
+        const float su = u[b] + u2[b], du = u[b] - u2[b], sw = w[b] + w2[b], dw = w[b] - w2[b];
+        A[lo] = 0.5f * (su - dw);
+        A[hi] = 0.5f * (su + dw);
+        B[lo] = 0.5f * (sw + du);
+        B[hi] = 0.5f * (sw - du);
+      } else {
+        A[lo] = u[b] - u2[b];
+        A[hi] = u[b] + u2[b];
+        B[lo] = 0.0f;
+        B[hi] = 0.0f;
+      }
     }
   }
 }
@@ -123,46 +169,71 @@ RD_HD void cols_orbit_pass(float* tile, int NR, int tid, int NT) {
 }
 
 // Forward, tile -> HBM: combine each pair into Re / Im of Y (see the top of the file).
-template <class G, int W, typename T>
-RD_HD void cols_store_fwd(const float* tile, T* img, int C, int k0, int tid, int NT) {
-  constexpr int R = G::P, H = W / 2;
-  for (int idx = tid; idx < R * W; idx += NT) {
-    const int r = idx / W, j = idx % W;
-    const int col = strip_col(j, H, k0, C);
-    if (col < 0) continue;
-    const int jl = j < H ? j : j - H;
-    const int k = k0 + jl;
-    float val;
-    if (k > 0 && k < C / 2 && r != 0 && r != R / 2) {
-      const float* A = tile + G::row_base(jl);
-      const float* B = tile + G::row_base(jl + H);
-      const int k1 = r < R / 2 ? r : R - r;
-      const float ar = A[G::at(k1)], ai = A[G::at(R - k1)];
-      const float br = B[G::at(k1)], bi = B[G::at(R - k1)];
-      if (j < H) val = r < R / 2 ? ar - bi : ar + bi;
-      else val = r < R / 2 ? ai + br : br - ai;
-    } else {
-      val = tile[G::row_base(j) + G::at(r)];
+// Thread tid owns left column k = k0 + tid % H (and its mirror) and the row pairs
+// (k1, R - k1), k1 = q0 + i STEP, as cols_load_unpair; k1 = 0 stands for (0, R/2).
+template <class G, int W, int NT, typename T>
+RD_HD void cols_store_fwd(const float* tile, T* img, int C, int k0, int tid) {
+  constexpr int R = G::P, H = W / 2, Q = R / 2, STEP = NT / H, ITER = Q / STEP;
+  const int jl = tid % H, q0 = tid / H;
+  const int k = k0 + jl;
+  if (k > C / 2) return;
+  const bool paired = k > 0 && k < C / 2;
+  const float* A = tile + G::row_base(jl);
+  const float* B = tile + G::row_base(jl + H);
+  T* ca = img + k;
+  T* cb = img + (paired ? C - k : 0);
+#pragma unroll 4
+  for (int i = 0; i < ITER; ++i) {
+    const int k1 = q0 + i * STEP;
+    const int rlo = k1, rhi = k1 == 0 ? Q : R - k1;
+    const float ar = A[G::at(rlo)], ai = A[G::at(rhi)];
+    if (!paired) {
+      ca[(int64_t)rlo * C] = from_f32<T>(ar);
+      ca[(int64_t)rhi * C] = from_f32<T>(ai);
+      continue;
     }
-    img[(int64_t)r * C + col] = from_f32<T>(val);
+    const float br = B[G::at(rlo)], bi = B[G::at(rhi)];
+    if (k1 == 0) {
+      ca[0] = from_f32<T>(ar);
+      ca[(int64_t)Q * C] = from_f32<T>(ai);
+      cb[0] = from_f32<T>(br);
+      cb[(int64_t)Q * C] = from_f32<T>(bi);
+    } else {
+      ca[(int64_t)rlo * C] = from_f32<T>(ar - bi);
+      ca[(int64_t)rhi * C] = from_f32<T>(ar + bi);
+      cb[(int64_t)rlo * C] = from_f32<T>(ai + br);
+      cb[(int64_t)rhi * C] = from_f32<T>(br - ai);
+    }
   }
 }
 
 // Inverse, tile -> HBM: the second mirror and the 1/R of the Hartley-form inverse.
-template <class G, int W, typename T>
-RD_HD void cols_store_inv(const float* tile, T* img, int C, int k0, int tid, int NT) {
-  constexpr int R = G::P, H = W / 2;
+// Thread tid owns tile row j = tid % W and the row pairs (k1, R - k1), k1 = q0 + i
+// STEP (q0 = tid / W, STEP = NT / W); k1 = 0 stands for (0, R/2).
+template <class G, int W, int NT, typename T>
+RD_HD void cols_store_inv(const float* tile, T* img, int C, int k0, int tid) {
+  constexpr int R = G::P, H = W / 2, Q = R / 2, STEP = NT / W, ITER = Q / STEP;
   constexpr float scale = 1.0f / R;
-  for (int idx = tid; idx < R * W; idx += NT) {
-    const int r = idx / W, j = idx % W;
-    const int col = strip_col(j, H, k0, C);
-    if (col < 0) continue;
-    const float* X = tile + G::row_base(j);
-    float val;
-    if (r == 0 || r == R / 2) val = X[G::at(r)] * scale;
-    else if (r < R / 2) val = (X[G::at(r)] - X[G::at(R - r)]) * scale;
-    else val = (X[G::at(R - r)] + X[G::at(r)]) * scale;
-    img[(int64_t)r * C + col] = from_f32<T>(val);
+  const int j = tid % W, q0 = tid / W;
+  const int col = strip_col(j, H, k0, C);
+  if (col < 0) return;
+  const float* X = tile + G::row_base(j);
+  T* dst = img + col;
+#pragma unroll 4
+  for (int i = 0; i < ITER; ++i) {
+    const int k1 = q0 + i * STEP;
+    const int rlo = k1, rhi = k1 == 0 ? Q : R - k1;
+    const float a = X[G::at(rlo)], b = X[G::at(rhi)];
+    float lo, hi;
+    if (k1 == 0) {
+      lo = a * scale;
+      hi = b * scale;
+    } else {
+      lo = (a - b) * scale;
+      hi = (a + b) * scale;
+    }
+    dst[(int64_t)rlo * C] = from_f32<T>(lo);
+    dst[(int64_t)rhi * C] = from_f32<T>(hi);
   }
 }
 

@@ -22,11 +22,10 @@ __device__ __forceinline__ void run_steps(float* tile, int lrow, int v, RowPtr r
   }
 }
 
-// One CTA: ROWS consecutive rows. For p >= 64 the rows travel between HBM and a
-// padded shared staging buffer by bulk copies (the TMA engine, no per-element load or
-// store instructions), and the passes read their first input from and write their
-// last output to that buffer. The pad (64 bytes per row) puts the two rows that share
-// a warp at p = 512 in opposite halves of the banks.
+// One CTA: ROWS consecutive rows. For p >= 64 the rows travel between HBM and the
+// staging buffer by bulk copies (the TMA engine, no per-element load or store
+// instructions), and the passes read their first input from and write their last
+// output to that buffer.
 template <int P, bool INV, typename T>
 __global__ void __launch_bounds__(RowTiling<P>::THREADS)
 k_rows(T* __restrict__ data, int64_t rows) {
@@ -36,34 +35,35 @@ k_rows(T* __restrict__ data, int64_t rows) {
     if (row < rows) row_small<P, INV, T>(data + row * P);
   } else {
     using G = RowGeo<P>;
+    using SM = RowSmem<P, T>;
     constexpr int TPR = G::TPR;
-    constexpr int RAW_ROW = P * (int)sizeof(T);
-    constexpr int RAW_STRIDE = RAW_ROW + 64;
-    __shared__ __align__(128) unsigned char raw[ROWS * RAW_STRIDE];
-    __shared__ float tile[G::words(ROWS)];
-    __shared__ __align__(8) uint64_t mbar;
+    extern __shared__ __align__(128) unsigned char smem[];
+    unsigned char* raw = smem;
+    float* tile = reinterpret_cast<float*>(smem + SM::TILE_OFF);
+    uint64_t* mbar = reinterpret_cast<uint64_t*>(smem + SM::MBAR_OFF);
     const int64_t row0 = (int64_t)blockIdx.x * ROWS;
     const int nr = (int)((rows - row0) < ROWS ? (rows - row0) : ROWS);
     if (threadIdx.x == 0) {
-      mbar_init(&mbar, 1);
-      mbar_arrive_expect_tx(&mbar, (unsigned)(nr * RAW_ROW));
-      for (int r = 0; r < nr; ++r) bulk_load(raw + r * RAW_STRIDE, data + (row0 + r) * P, RAW_ROW, &mbar);
+      mbar_init(mbar, 1);
+      mbar_arrive_expect_tx(mbar, (unsigned)(nr * SM::RAW_ROW));
+      for (int r = 0; r < nr; ++r)
+        bulk_load(raw + SM::raw_off(r), data + (row0 + r) * P, SM::RAW_ROW, mbar);
     }
     __syncthreads();                                  // the barrier exists before anyone waits
-    const bool arrived = mbar_wait_bounded(&mbar, 0);
+    const bool arrived = mbar_wait_bounded(mbar, 0);
     if (!__syncthreads_and(arrived)) {
-      mbar_wait_bounded(&mbar, 0);                    // give copies in flight a last chance
+      mbar_wait_bounded(mbar, 0);                     // give copies in flight a last chance
       return;
     }
     const int lrow = threadIdx.x / TPR;
     const int v = threadIdx.x % TPR;
     auto rowok = [&](int r) { return r < nr; };
-    auto rowptr = [&](int r) { return reinterpret_cast<T*>(raw + r * RAW_STRIDE); };
+    auto rowptr = [&](int r) { return reinterpret_cast<T*>(raw + SM::raw_off(r)); };
     run_steps<G, INV, 0, ROWS, T>(tile, lrow, v, rowptr, rowok);
     fence_smem_to_async();
     __syncthreads();
     if (threadIdx.x == 0) {
-      for (int r = 0; r < nr; ++r) bulk_store(data + (row0 + r) * P, raw + r * RAW_STRIDE, RAW_ROW);
+      for (int r = 0; r < nr; ++r) bulk_store(data + (row0 + r) * P, raw + SM::raw_off(r), SM::RAW_ROW);
       bulk_commit();
       bulk_wait_all();
     }
@@ -91,15 +91,28 @@ cudaError_t launch_wait_selftest(cudaStream_t s) {
   return cudaGetLastError();
 }
 
-template <int P, typename T>
-static cudaError_t launch_p(void* data, int64_t rows, bool inverse, cudaStream_t s) {
+template <int P, bool INV, typename T>
+static cudaError_t launch_pi(T* d, int64_t rows, cudaStream_t s) {
   constexpr int ROWS = RowTiling<P>::ROWS;
   const int64_t grid = (rows + ROWS - 1) / ROWS;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  T* d = static_cast<T*>(data);
-  if (inverse) k_rows<P, true, T><<<(unsigned)grid, RowTiling<P>::THREADS, 0, s>>>(d, rows);
-  else k_rows<P, false, T><<<(unsigned)grid, RowTiling<P>::THREADS, 0, s>>>(d, rows);
+  size_t smem = 0;
+  if constexpr (P > 32) {
+    smem = RowSmem<P, T>::BYTES;
+    if (smem > 48 * 1024) {
+      const cudaError_t e = cudaFuncSetAttribute(k_rows<P, INV, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+  }
+  k_rows<P, INV, T><<<(unsigned)grid, RowTiling<P>::THREADS, smem, s>>>(d, rows);
   return cudaGetLastError();
+}
+
+template <int P, typename T>
+static cudaError_t launch_p(void* data, int64_t rows, bool inverse, cudaStream_t s) {
+  T* d = static_cast<T*>(data);
+  return inverse ? launch_pi<P, true, T>(d, rows, s) : launch_pi<P, false, T>(d, rows, s);
 }
 
 template <typename T>

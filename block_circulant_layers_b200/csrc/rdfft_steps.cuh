@@ -61,12 +61,36 @@ RD_HD void row_small(T* g) {
   }
 }
 
-// Rows per CTA: 32 threads (two rows) at p = 512, 128 threads otherwise (measured best
-// on B200 among 32..256 threads); 128 rows of one thread each for p <= 32.
+// Rows per CTA: 128 threads (8 rows at p = 512, one at p = 4096), measured best on
+// B200 among 32..512 threads with the bulk-copy staging (wider CTAs put more rows'
+// merged orbits in one warp, narrower ones wait less at barriers); 128 rows of one
+// thread each for p <= 32.
 template <int P>
 struct RowTiling {
-  static constexpr int THREADS = P == 512 ? 32 : 128;
+  static constexpr int THREADS = 128;
   static constexpr int ROWS = (P <= 32) ? THREADS : THREADS / RowGeo<P>::TPR;
+};
+
+// Shared-memory plan of a rows CTA (p >= 64), dynamic: the staging buffer of the
+// rows as they are in HBM, the fp32 tile, the mbarrier. A step of pass 0 has the
+// TPR lanes of a row read TPR consecutive elements (SEG bytes, at least 16), and the
+// RW rows of a warp read at once; staged row r starts at r (RAW_ROW + SEG) +
+// 16 (r / RW) bytes. So staged rows are 16-byte aligned for the bulk copies and never
+// overlap, the RW rows of a warp read disjoint banks, and consecutive warp groups are
+// shifted by one more 16-byte bank group (for the merged orbits, which one warp
+// stores for many rows at the same in-row position).
+template <int P, typename T>
+struct RowSmem {
+  static constexpr int ROWS = RowTiling<P>::ROWS;
+  static constexpr int TPR = RowGeo<P>::TPR;
+  static constexpr int RW = TPR < 32 ? 32 / TPR : 1;
+  static constexpr int RAW_ROW = P * (int)sizeof(T);
+  static constexpr int SEG = TPR * (int)sizeof(T) < 16 ? 16 : TPR * (int)sizeof(T);
+  RD_HD static constexpr int raw_off(int r) { return r * (RAW_ROW + SEG) + 16 * (r / RW); }
+  static constexpr int TILE_OFF = raw_off(ROWS - 1) + RAW_ROW;
+  static constexpr int MBAR_OFF = TILE_OFF + ((RowGeo<P>::words(ROWS) * 4 + 15) / 16) * 16;
+  static constexpr int BYTES = MBAR_OFF + 16;
+  static_assert(RAW_ROW % 16 == 0 && SEG % 16 == 0 && TILE_OFF % 16 == 0, "16-byte alignment");
 };
 
 }  // namespace rdfft

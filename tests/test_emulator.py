@@ -151,3 +151,32 @@ def test_hartley_form_inverse_matches_oracle(emu, p):
     assert emu.rdfft_emulate_hartley_inverse(a.ctypes.data, rows, p, 0) == 0
     ref = oracle.idft_packed(s.exact)
     assert np.abs(a - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("dtype", [0, 1])
+@pytest.mark.parametrize("p", [64, 128, 256, 512, 1024, 2048, 4096])
+def test_rows_kernel_shared_memory_plan(emu, p, dtype):
+    """The rows kernel's shared-memory plan: staged rows 16-byte aligned (bulk copies),
+    disjoint, below the tile, the tile below the mbarrier, all within the 227 KiB a CTA
+    may have; the first step of pass 0 (the RW rows of a warp, TPR lanes each, reading
+    consecutive elements) conflict-free in the 32 four-byte banks from p = 128 on."""
+    emu.rdfft_row_smem_plan.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
+    out = (ctypes.c_int64 * 7000)()
+    assert emu.rdfft_row_smem_plan(p, dtype, out) == 0
+    rows, raw_row, tile_off, mbar_off, total, words, tpr = (int(out[i]) for i in range(7))
+    offs = [int(out[7 + r]) for r in range(rows)]
+    esz = 4 if dtype == 0 else 2
+    assert raw_row == p * esz
+    assert all(o % 16 == 0 for o in offs) and tile_off % 16 == 0 and mbar_off % 8 == 0
+    assert all(offs[r + 1] >= offs[r] + raw_row for r in range(rows - 1))
+    assert offs[-1] + raw_row <= tile_off and tile_off + 4 * words <= mbar_off and mbar_off + 8 <= total
+    assert total <= 227 * 1024
+    rw = max(32 // tpr, 1)
+    for g in range(0, rows, rw):
+        banks = {}
+        for r in range(g, min(g + rw, rows)):
+            for v in range(min(tpr, 32)):
+                word = (offs[r] + v * esz) // 4
+                banks.setdefault(word % 32, set()).add(word)
+        worst = max(len(ws) for ws in banks.values())
+        assert worst <= (2 if p == 64 else 1), (p, dtype, worst)
