@@ -43,19 +43,22 @@ POOL = 64                   # tensors per view; 2 MiB each in bf16
 STREAMS = 8
 FALLBACK_HBM_GBS = 6650.0
 
+ROWS_KERNEL_SOURCES = ("bulk_copy.cuh", "gen_twiddles.py", "packed_fft.cuh", "rdfft_kernels.cu", "rdfft_steps.cuh")
+
 # ncu dram bytes per launch of the dominant kernel, with the hash of the kernel
 # sources they were captured from (see profiles/); stale counters are reported null.
-TRAFFIC_CAPTURE = {"sources_sha1": None, "kernel": None, "bytes_per_launch": None}
+TRAFFIC_CAPTURE = {"sources_sha1": "3332b8c137a2c930ea36fe877b18e31d046142cf", "kernel": "bf16_p4096_inv",
+                   "bytes_per_launch": 3451766}
 
 
 def kernel_sources_sha1() -> str:
+    """Hash of the sources of the rows kernel (the bench step's only kernel)."""
     h = hashlib.sha1()
     csrc = os.path.join(ROOT, "block_circulant_layers_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
-        if name.endswith((".cu", ".cuh", ".h", ".py")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode())
-                h.update(f.read())
+    for name in ROWS_KERNEL_SOURCES:
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode())
+            h.update(f.read())
     return h.hexdigest()
 
 

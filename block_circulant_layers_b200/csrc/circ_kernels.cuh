@@ -136,7 +136,7 @@ __device__ __forceinline__ int bin_im_slot(int k) { return k == 0 ? P / 2 : P - 
 // BWDX = true : in = g, out = grad_x; the CTA's QI output blocks are j, summed over i,
 //               against conj(c_hat).
 template <int P, typename T, int NT, int TT, int NS, bool BWDX>
-__global__ void __launch_bounds__(NT)
+__global__ void __launch_bounds__(NT, NT >= 256 ? 2 : 1)   // 256-thread CTAs: two per SM (<= 128 registers)
 k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict__ out,
          int64_t B, int q, int QI) {
   extern __shared__ float tile[];
