@@ -163,6 +163,93 @@ RD_HD void bfly(float& pk, float& pmk, float& pHk, float& pMk, Tw w) {
   else bfly_fwd(pk, pmk, pHk, pMk, w.c, -w.s);
 }
 
+// ------------------------------------------------------------------ paired stages
+// sm_100 executes two fp32 FMAs, adds or multiplies in one instruction on a float2
+// register pair. Every stage but the last of a register block applies the same
+// operations and twiddles to both halves of the block, so those stages run on pairs
+// (a[i], a[i + HALF]). Each packed operation rounds exactly like the scalar one it
+// replaces (a - b is fma(b, -1, a); 2e - a is fma(a, -1, e + e)), so the results are
+// bit-identical to the scalar butterflies above.
+#if defined(__CUDA_ARCH__)
+typedef float2 f2;
+RD_HD f2 f2_mk(float x, float y) { return make_float2(x, y); }
+RD_HD f2 f2_fma(f2 a, f2 b, f2 c) { return __ffma2_rn(a, b, c); }
+RD_HD f2 f2_add(f2 a, f2 b) { return __fadd2_rn(a, b); }
+RD_HD f2 f2_mul(f2 a, f2 b) { return __fmul2_rn(a, b); }
+#else
+struct f2 { float x, y; };
+RD_HD f2 f2_mk(float x, float y) { return f2{x, y}; }
+RD_HD f2 f2_fma(f2 a, f2 b, f2 c) { return f2{fmaf(a.x, b.x, c.x), fmaf(a.y, b.y, c.y)}; }
+RD_HD f2 f2_add(f2 a, f2 b) { return f2{a.x + b.x, a.y + b.y}; }
+RD_HD f2 f2_mul(f2 a, f2 b) { return f2{a.x * b.x, a.y * b.y}; }
+#endif
+RD_HD f2 f2_bc(float v) { return f2_mk(v, v); }
+RD_HD f2 f2_sub(f2 a, f2 b) { return f2_fma(b, f2_bc(-1.0f), a); }
+
+// bfly_fwd on two groups at once (nwi = -wi).
+RD_HD void bfly_fwd2(f2& pk, f2& pmk, f2& pHk, f2& pMk, f2 wr, f2 wi, f2 nwi) {
+  const f2 er = pk, ei = pmk, orr = pHk, oi = pMk;
+  const f2 ar = f2_fma(wr, orr, f2_fma(nwi, oi, er));
+  const f2 ai = f2_fma(wr, oi, f2_fma(wi, orr, ei));
+  pk = ar;
+  pMk = ai;
+  pmk = f2_fma(ar, f2_bc(-1.0f), f2_add(er, er));
+  pHk = f2_fma(f2_bc(-2.0f), ei, ai);
+}
+
+// bfly_inv on two groups at once (nwi = -wi).
+RD_HD void bfly_inv2(f2& pk, f2& pmk, f2& pHk, f2& pMk, f2 wr, f2 wi, f2 nwi) {
+  const f2 a = pk, b = pMk, c = pmk, d = pHk;
+  const f2 dr = f2_sub(a, c), di = f2_add(b, d);
+  pk = f2_add(a, c);
+  pmk = f2_sub(b, d);
+  pHk = f2_fma(dr, wr, f2_mul(di, wi));
+  pMk = f2_fma(di, wr, f2_mul(dr, nwi));
+}
+
+// The group (i0, i1, i2, i3) of the lower half and the same group of the upper half
+// (+HALF) as one paired butterfly with twiddle w.
+template <bool INV, int HALF, int E>
+RD_HD void bfly_pair(float (&a)[E], int i0, int i1, int i2, int i3, Tw w) {
+  f2 x0 = f2_mk(a[i0], a[i0 + HALF]), x1 = f2_mk(a[i1], a[i1 + HALF]);
+  f2 x2 = f2_mk(a[i2], a[i2 + HALF]), x3 = f2_mk(a[i3], a[i3 + HALF]);
+  const f2 wr = f2_bc(w.c), wi = f2_bc(-w.s), nwi = f2_bc(w.s);
+  if (INV) bfly_inv2(x0, x1, x2, x3, wr, wi, nwi);
+  else bfly_fwd2(x0, x1, x2, x3, wr, wi, nwi);
+  a[i0] = x0.x; a[i0 + HALF] = x0.y;
+  a[i1] = x1.x; a[i1 + HALF] = x1.y;
+  a[i2] = x2.x; a[i2 + HALF] = x2.y;
+  a[i3] = x3.x; a[i3 + HALF] = x3.y;
+}
+
+// Stage M on the blocks of a[OFF, OFF + HALF) and, identically, of the upper half.
+template <int M, int HALF, int OFF, bool INV, int E>
+RD_HD void stage_paired(float (&a)[E]) {
+  static_assert(HALF % M == 0 && OFF + 2 * HALF <= E, "paired stage range");
+#pragma unroll
+  for (int b = OFF; b < OFF + HALF; b += M) {
+    const f2 x0 = f2_mk(a[b], a[b + HALF]), x1 = f2_mk(a[b + M / 2], a[b + M / 2 + HALF]);
+    const f2 s = f2_add(x0, x1), d = f2_sub(x0, x1);
+    a[b] = s.x; a[b + HALF] = s.y;
+    a[b + M / 2] = d.x; a[b + M / 2 + HALF] = d.y;
+    if (M >= 4) {
+      constexpr int q1 = M / 4, q3 = 3 * M / 4;
+      if (INV) {
+        const f2 y1 = f2_mul(f2_mk(a[b + q1], a[b + q1 + HALF]), f2_bc(2.0f));
+        const f2 y3 = f2_mul(f2_mk(a[b + q3], a[b + q3 + HALF]), f2_bc(-2.0f));
+        a[b + q1] = y1.x; a[b + q1 + HALF] = y1.y;
+        a[b + q3] = y3.x; a[b + q3 + HALF] = y3.y;
+      } else {
+        const f2 y3 = f2_mul(f2_mk(a[b + q3], a[b + q3 + HALF]), f2_bc(-1.0f));
+        a[b + q3] = y3.x; a[b + q3 + HALF] = y3.y;
+      }
+    }
+#pragma unroll
+    for (int k = 1; k < M / 4; ++k)
+      bfly_pair<INV, HALF>(a, b + k, b + M / 2 - k, b + M / 2 + k, b + M - k, tw_const(tw_index(M, k)));
+  }
+}
+
 // One stage of size M over the contiguous register range a[OFF, OFF + NB).
 // The positions are the algorithm's own; twiddles are compile-time.
 template <int M, int NB, int OFF, bool INV, int E>
@@ -189,14 +276,21 @@ RD_HD void stage_contig(float (&a)[E]) {
 
 // Stages MLO..MHI (powers of two) on a[OFF, OFF+NB): ascending for the forward
 // transform, descending for the inverse.
+// Stage M of a block of NB registers: on pairs while M <= NB/2, else scalar.
+template <int M, int NB, int OFF, bool INV, int E>
+RD_HD void stage_block(float (&a)[E]) {
+  if constexpr (M <= NB / 2) stage_paired<M, NB / 2, OFF, INV>(a);
+  else stage_contig<M, NB, OFF, INV>(a);
+}
+
 template <int MLO, int MHI, int NB, int OFF, bool INV, int E>
 RD_HD void stages_contig(float (&a)[E]) {
   if constexpr (MLO <= MHI) {
     if constexpr (!INV) {
-      stage_contig<MLO, NB, OFF, false>(a);
+      stage_block<MLO, NB, OFF, false>(a);
       stages_contig<MLO * 2, MHI, NB, OFF, false>(a);
     } else {
-      stage_contig<MHI, NB, OFF, true>(a);
+      stage_block<MHI, NB, OFF, true>(a);
       stages_contig<MLO, MHI / 2, NB, OFF, true>(a);
     }
   }
@@ -230,15 +324,50 @@ RD_HD void orbit_stage(float (&a)[E], int r) {
   }
 }
 
+// Stage U <= UMAX/2 of a generic orbit on pairs: block m0 of the lower half of the
+// orbit (m < UMAX/2, elements OFF .. OFF + UMAX) with block m0 + UMAX/2 (elements
+// + UMAX), which takes the same twiddles.
+template <int H, int UMAX, int U, int OFF, bool INV, int E>
+RD_HD void orbit_stage_paired(float (&a)[E], int r) {
+  constexpr int MP = U * H;
+  constexpr int U2 = U / 2;
+  constexpr int HALF = UMAX;
+  if constexpr (U == 2) {
+    const Tw w = tw_lane(tw_index(MP, 0) + r);
+#pragma unroll
+    for (int m0 = 0; m0 < UMAX / 2; m0 += 2)
+      bfly_pair<INV, HALF>(a, OFF + 2 * m0, OFF + 2 * m0 + 1, OFF + 2 * m0 + 2, OFF + 2 * m0 + 3, w);
+  } else {
+#pragma unroll
+    for (int s = 0; s < U / 4; ++s) {
+      const Tw w1 = tw_lane(tw_index(MP, s * H) + r);
+      const Tw w2 = tw_lane(tw_index(MP, (s + 1) * H) - r);
+#pragma unroll
+      for (int m0 = 0; m0 < UMAX / 2; m0 += U) {
+        bfly_pair<INV, HALF>(a, OFF + 2 * (m0 + s), OFF + 2 * (m0 + U2 - s - 1) + 1, OFF + 2 * (m0 + U2 + s),
+                             OFF + 2 * (m0 + U - s - 1) + 1, w1);
+        bfly_pair<INV, HALF>(a, OFF + 2 * (m0 + s) + 1, OFF + 2 * (m0 + U2 - s - 1), OFF + 2 * (m0 + U2 + s) + 1,
+                             OFF + 2 * (m0 + U - s - 1), w2);
+      }
+    }
+  }
+}
+
+template <int H, int UMAX, int U, int OFF, bool INV, int E>
+RD_HD void orbit_stage_any(float (&a)[E], int r) {
+  if constexpr (U <= UMAX / 2) orbit_stage_paired<H, UMAX, U, OFF, INV>(a, r);
+  else orbit_stage<H, UMAX, U, OFF, INV>(a, r);
+}
+
 template <int H, int UMAX, int U, int OFF, bool INV, int E>
 RD_HD void orbit_stages(float (&a)[E], int r) {
   if constexpr (U <= UMAX) {
     if constexpr (!INV) {
-      orbit_stage<H, UMAX, U, OFF, false>(a, r);
+      orbit_stage_any<H, UMAX, U, OFF, false>(a, r);
       orbit_stages<H, UMAX, U * 2, OFF, false>(a, r);
     } else {
       orbit_stages<H, UMAX, U * 2, OFF, true>(a, r);
-      orbit_stage<H, UMAX, U, OFF, true>(a, r);
+      orbit_stage_any<H, UMAX, U, OFF, true>(a, r);
     }
   }
 }
