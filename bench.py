@@ -47,8 +47,8 @@ ROWS_KERNEL_SOURCES = ("bulk_copy.cuh", "gen_twiddles.py", "packed_fft.cuh", "rd
 
 # ncu dram bytes per launch of the dominant kernel, with the hash of the kernel
 # sources they were captured from (see profiles/); stale counters are reported null.
-TRAFFIC_CAPTURE = {"sources_sha1": "3332b8c137a2c930ea36fe877b18e31d046142cf", "kernel": "bf16_p4096_inv",
-                   "bytes_per_launch": 3451766}
+TRAFFIC_CAPTURE = {"sources_sha1": "4f14a0c2aafddc272516c8ae361467179ec6a51e",
+                   "bytes_per_launch": {"bf16_p4096_inv": 3446845, "bf16_p4096_fwd": 3452154}}
 
 
 def kernel_sources_sha1() -> str:
@@ -375,8 +375,8 @@ def run_ours(args):
     achieved = bytes_per_transform / (dom["us_per_launch_amortized"] * 1e-6) / 1e9
     srcs = kernel_sources_sha1()
     traffic = None
-    if TRAFFIC_CAPTURE["sources_sha1"] == srcs and TRAFFIC_CAPTURE["kernel"] == dom_key:
-        traffic = TRAFFIC_CAPTURE["bytes_per_launch"]
+    if TRAFFIC_CAPTURE["sources_sha1"] == srcs:
+        traffic = TRAFFIC_CAPTURE["bytes_per_launch"].get(dom_key)
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
                 "frac": round(achieved / hbm_peak, 4), "traffic": traffic, "kernel": dom_key,
                 "peak_kind": peak_kind,
