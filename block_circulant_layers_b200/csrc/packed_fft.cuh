@@ -296,6 +296,34 @@ RD_HD void stages_contig(float (&a)[E]) {
   }
 }
 
+// Twiddles of orbit stage U (M' = U*H) for s < U/4 from one loaded value
+// B = W_M'^r: W_M'^(s*H + r) = W_U^s * B and W_M'^((s+1)*H - r) = W_U^(s+1) * conj(B),
+// with W_U^s compile-time; W_U^0 = 1 and W_U^(U/4) = -i make those cases exact. So a
+// stage loads one lane-dependent twiddle instead of U/2 (Tw {c, s} is c - i s).
+template <int U, int S>
+RD_HD void orbit_twiddles(Tw B, Tw& w1, Tw& w2) {
+  if constexpr (S == 0) {
+    w1 = B;
+  } else {
+    const Tw c = tw_const(tw_index(U, S));
+    w1 = Tw{fmaf(c.c, B.c, -(c.s * B.s)), fmaf(c.c, B.s, c.s * B.c)};
+  }
+  if constexpr (S + 1 == U / 4) {
+    w2 = Tw{B.s, B.c};
+  } else {
+    const Tw d = tw_const(tw_index(U, S + 1));
+    w2 = Tw{fmaf(d.c, B.c, d.s * B.s), fmaf(d.s, B.c, -(d.c * B.s))};
+  }
+}
+
+template <int U, int S = 0>
+RD_HD void orbit_stage_twiddles(int s, Tw B, Tw& w1, Tw& w2) {
+  if constexpr (S < U / 4) {
+    if (s == S) orbit_twiddles<U, S>(B, w1, w2);
+    else orbit_stage_twiddles<U, S + 1>(s, B, w1, w2);
+  }
+}
+
 // Generic orbit: a[OFF + 2m] <-> position m*H + r, a[OFF + 2m + 1] <-> (m+1)*H - r,
 // m < UMAX. Stage M' = U*H (U = 2..UMAX) acts on the groups with k' = s*H + r and
 // k' = (s+1)*H - r (s < U/4), or k' = r alone when U = 2.
@@ -309,10 +337,11 @@ RD_HD void orbit_stage(float (&a)[E], int r) {
     for (int m0 = 0; m0 < UMAX; m0 += 2)
       bfly<INV>(a[OFF + 2 * m0], a[OFF + 2 * m0 + 1], a[OFF + 2 * m0 + 2], a[OFF + 2 * m0 + 3], w);
   } else {
+    const Tw B = tw_lane(tw_index(MP, 0) + r);
 #pragma unroll
     for (int s = 0; s < U / 4; ++s) {
-      const Tw w1 = tw_lane(tw_index(MP, s * H) + r);
-      const Tw w2 = tw_lane(tw_index(MP, (s + 1) * H) - r);
+      Tw w1, w2;
+      orbit_stage_twiddles<U>(s, B, w1, w2);
 #pragma unroll
       for (int m0 = 0; m0 < UMAX; m0 += U) {
         bfly<INV>(a[OFF + 2 * (m0 + s)], a[OFF + 2 * (m0 + U2 - s - 1) + 1],
@@ -338,10 +367,11 @@ RD_HD void orbit_stage_paired(float (&a)[E], int r) {
     for (int m0 = 0; m0 < UMAX / 2; m0 += 2)
       bfly_pair<INV, HALF>(a, OFF + 2 * m0, OFF + 2 * m0 + 1, OFF + 2 * m0 + 2, OFF + 2 * m0 + 3, w);
   } else {
+    const Tw B = tw_lane(tw_index(MP, 0) + r);
 #pragma unroll
     for (int s = 0; s < U / 4; ++s) {
-      const Tw w1 = tw_lane(tw_index(MP, s * H) + r);
-      const Tw w2 = tw_lane(tw_index(MP, (s + 1) * H) - r);
+      Tw w1, w2;
+      orbit_stage_twiddles<U>(s, B, w1, w2);
 #pragma unroll
       for (int m0 = 0; m0 < UMAX / 2; m0 += U) {
         bfly_pair<INV, HALF>(a, OFF + 2 * (m0 + s), OFF + 2 * (m0 + U2 - s - 1) + 1, OFF + 2 * (m0 + U2 + s),
