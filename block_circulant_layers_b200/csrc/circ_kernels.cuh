@@ -152,84 +152,178 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
   });
   __syncthreads();
 
-  // 2. contraction: thread slot s covers bin k and output block ol of all TT tokens
-  constexpr int HB = P / 2;
-  float acc_r[NS][TT], acc_i[NS][TT];
-#pragma unroll
-  for (int s = 0; s < NS; ++s)
-#pragma unroll
-    for (int t = 0; t < TT; ++t) acc_r[s][t] = acc_i[s][t] = 0.0f;
+  // 2.-3. contraction and output spectra. When all of a thread's slots share one bin
+  // (NT a multiple of p/2, i.e. p <= 512), slot pairs run on packed fp32 pairs; with a
+  // bin per slot (p >= 1024) pairing saves no loads and costs registers, so it is scalar.
+  if constexpr (NT % (P / 2) == 0 && NS >= 2) {
+    // 2. contraction: thread slot s covers bin k and output block ol of all TT tokens.
+    // Slots are taken in pairs (s, s + 1) on packed fp32 pairs: each pair accumulates
+    // two output blocks (two bins at p >= 1024) of one token in one FFMA2 per term.
+    constexpr int HB = P / 2;
+    constexpr int NP = (NS + 1) / 2;              // slot pairs (an odd last slot pairs with a zero slot)
+    f2 acc_r[NP][TT], acc_i[NP][TT];
+  #pragma unroll
+    for (int u = 0; u < NP; ++u)
+  #pragma unroll
+      for (int t = 0; t < TT; ++t) acc_r[u][t] = acc_i[u][t] = f2_bc(0.0f);
 
-  // c_hat of the summed block j + 1 is loaded (through L2) while block j is
-  // contracted, so the L2 latency overlaps the FMA work.
-  float cr_n[NS], ci_n[NS];
-  auto load_c = [&](int j, float (&cr)[NS], float (&ci)[NS]) {
-#pragma unroll
+    // c_hat of the summed block j + 1 is loaded (through L2) while block j is
+    // contracted, so the L2 latency overlaps the FMA work.
+    float cr_n[2 * NP], ci_n[2 * NP];
+    auto load_c = [&](int j, float (&cr)[2 * NP], float (&ci)[2 * NP]) {
+  #pragma unroll
+      for (int s = 0; s < 2 * NP; ++s) {
+        const int pi = threadIdx.x + NT * s;
+        const int ol = pi / HB, k = pi % HB;
+        if (s < NS && ol < QI) {
+          const int ob = o0 + ol;
+          const float* crow = chat + (int64_t)(BWDX ? (j * q + ob) : (ob * q + j)) * P;
+          cr[s] = __ldg(crow + k);
+          ci[s] = __ldg(crow + bin_im_slot<P>(k));
+        } else {
+          cr[s] = ci[s] = 0.0f;
+        }
+      }
+    };
+    load_c(0, cr_n, ci_n);
+    for (int j = 0; j < q; ++j) {                 // j: summed block (input j for fwd, output i for grad_x)
+      float cr_c[2 * NP], ci_c[2 * NP];
+  #pragma unroll
+      for (int sl = 0; sl < 2 * NP; ++sl) {
+        cr_c[sl] = cr_n[sl];
+        ci_c[sl] = ci_n[sl];
+      }
+      if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
+      // no guard on the slot here: a slot beyond the CTA's blocks has c = 0 (load_c), so
+      // its accumulators stay 0 and are never stored; slots that share a bin (all of
+      // them when NT >= p/2) share the loads of X.
+  #pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        const int rb = LayerGeo<P>::row_base(t * q + j);
+  #pragma unroll
+        for (int u = 0; u < NP; ++u) {
+          const int k0 = (threadIdx.x + NT * (2 * u)) % HB, k1 = (threadIdx.x + NT * (2 * u + 1)) % HB;
+          // packed product: bin 0 multiplies the real pair component-wise, other bins are
+          // complex products (conjugated c for grad_x):
+          //   acc_r += cr xr + a2 xi,  acc_i += a3 xi + a4 xr
+          const float ci0 = ci_c[2 * u], ci1 = ci_c[2 * u + 1];
+          const bool z0 = (k0 == 0), z1 = (k1 == 0);
+          const f2 c1 = f2_mk(cr_c[2 * u], cr_c[2 * u + 1]);
+          const f2 c2 = f2_mk(z0 ? 0.0f : (BWDX ? ci0 : -ci0), z1 ? 0.0f : (BWDX ? ci1 : -ci1));
+          const f2 c3 = f2_mk(z0 ? ci0 : cr_c[2 * u], z1 ? ci1 : cr_c[2 * u + 1]);
+          const f2 c4 = f2_mk(z0 ? 0.0f : (BWDX ? -ci0 : ci0), z1 ? 0.0f : (BWDX ? -ci1 : ci1));
+          const f2 xr = f2_mk(tile[rb + LayerGeo<P>::at(k0)], tile[rb + LayerGeo<P>::at(k1)]);
+          const f2 xi = f2_mk(tile[rb + LayerGeo<P>::at(bin_im_slot<P>(k0))],
+                              tile[rb + LayerGeo<P>::at(bin_im_slot<P>(k1))]);
+          acc_r[u][t] = f2_fma(c1, xr, f2_fma(c2, xi, acc_r[u][t]));
+          acc_i[u][t] = f2_fma(c3, xi, f2_fma(c4, xr, acc_i[u][t]));
+        }
+      }
+    }
+    __syncthreads();
+
+    // 3. output spectra over the tile: row t*QI + ol
+  #pragma unroll
     for (int s = 0; s < NS; ++s) {
       const int pi = threadIdx.x + NT * s;
       const int ol = pi / HB, k = pi % HB;
       if (ol < QI) {
-        const int ob = o0 + ol;
-        const float* crow = chat + (int64_t)(BWDX ? (j * q + ob) : (ob * q + j)) * P;
-        cr[s] = __ldg(crow + k);
-        ci[s] = __ldg(crow + bin_im_slot<P>(k));
-      } else {
-        cr[s] = ci[s] = 0.0f;
+        const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
+  #pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          // stored mirrored (slot k = Re - Im, slot p-k = Re + Im) for the Hartley-form
+          // inverse below; bin 0 keeps its real pair
+          const float ar = (s & 1) ? acc_r[s / 2][t].y : acc_r[s / 2][t].x;
+          const float ai = (s & 1) ? acc_i[s / 2][t].y : acc_i[s / 2][t].x;
+          const int rb = LayerGeo<P>::row_base(t * QI + ol);
+          tile[rb + kr] = k == 0 ? ar : ar - ai;
+          tile[rb + ki] = k == 0 ? ai : ar + ai;
+        }
       }
     }
-  };
-  load_c(0, cr_n, ci_n);
-  for (int j = 0; j < q; ++j) {                 // j: summed block (input j for fwd, output i for grad_x)
-    float cr_c[NS], ci_c[NS];
-#pragma unroll
-    for (int s = 0; s < NS; ++s) {
-      cr_c[s] = cr_n[s];
-      ci_c[s] = ci_n[s];
-    }
-    if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
-    // no guard on the slot here: a slot beyond the CTA's blocks has c = 0 (load_c), so
-    // its accumulators stay 0 and are never stored; without a branch, slots that share
-    // a bin (all of them when NT >= p/2) share the loads of X.
-#pragma unroll
-    for (int t = 0; t < TT; ++t) {
-      const int rb = LayerGeo<P>::row_base(t * q + j);
-#pragma unroll
-      for (int s = 0; s < NS; ++s) {
-        const int k = (threadIdx.x + NT * s) % HB;
-        const float cr = cr_c[s], ci = ci_c[s];
-        // packed product: bin 0 multiplies the real pair component-wise, other bins
-        // are complex products (conjugated c for grad_x)
-        const bool z = (k == 0);
-        const float a2 = z ? 0.0f : (BWDX ? ci : -ci);
-        const float a3 = z ? ci : cr;
-        const float a4 = z ? 0.0f : (BWDX ? -ci : ci);
-        const float xr = tile[rb + LayerGeo<P>::at(k)];
-        const float xi = tile[rb + LayerGeo<P>::at(bin_im_slot<P>(k))];
-        acc_r[s][t] = fmaf(cr, xr, fmaf(a2, xi, acc_r[s][t]));
-        acc_i[s][t] = fmaf(a3, xi, fmaf(a4, xr, acc_i[s][t]));
-      }
-    }
-  }
-  __syncthreads();
+    __syncthreads();
 
-  // 3. output spectra over the tile: row t*QI + ol
-#pragma unroll
-  for (int s = 0; s < NS; ++s) {
-    const int pi = threadIdx.x + NT * s;
-    const int ol = pi / HB, k = pi % HB;
-    if (ol < QI) {
-      const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
-#pragma unroll
+  } else {
+    // 2. contraction: thread slot s covers bin k and output block ol of all TT tokens
+    constexpr int HB = P / 2;
+    float acc_r[NS][TT], acc_i[NS][TT];
+  #pragma unroll
+    for (int s = 0; s < NS; ++s)
+  #pragma unroll
+      for (int t = 0; t < TT; ++t) acc_r[s][t] = acc_i[s][t] = 0.0f;
+
+    // c_hat of the summed block j + 1 is loaded (through L2) while block j is
+    // contracted, so the L2 latency overlaps the FMA work.
+    float cr_n[NS], ci_n[NS];
+    auto load_c = [&](int j, float (&cr)[NS], float (&ci)[NS]) {
+  #pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        const int pi = threadIdx.x + NT * s;
+        const int ol = pi / HB, k = pi % HB;
+        if (ol < QI) {
+          const int ob = o0 + ol;
+          const float* crow = chat + (int64_t)(BWDX ? (j * q + ob) : (ob * q + j)) * P;
+          cr[s] = __ldg(crow + k);
+          ci[s] = __ldg(crow + bin_im_slot<P>(k));
+        } else {
+          cr[s] = ci[s] = 0.0f;
+        }
+      }
+    };
+    load_c(0, cr_n, ci_n);
+    for (int j = 0; j < q; ++j) {                 // j: summed block (input j for fwd, output i for grad_x)
+      float cr_c[NS], ci_c[NS];
+  #pragma unroll
+      for (int s = 0; s < NS; ++s) {
+        cr_c[s] = cr_n[s];
+        ci_c[s] = ci_n[s];
+      }
+      if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
+      // no guard on the slot here: a slot beyond the CTA's blocks has c = 0 (load_c), so
+      // its accumulators stay 0 and are never stored; without a branch, slots that share
+      // a bin (all of them when NT >= p/2) share the loads of X.
+  #pragma unroll
       for (int t = 0; t < TT; ++t) {
-        // stored mirrored (slot k = Re - Im, slot p-k = Re + Im) for the Hartley-form
-        // inverse below; bin 0 keeps its real pair
-        const int rb = LayerGeo<P>::row_base(t * QI + ol);
-        tile[rb + kr] = k == 0 ? acc_r[s][t] : acc_r[s][t] - acc_i[s][t];
-        tile[rb + ki] = k == 0 ? acc_i[s][t] : acc_r[s][t] + acc_i[s][t];
+        const int rb = LayerGeo<P>::row_base(t * q + j);
+  #pragma unroll
+        for (int s = 0; s < NS; ++s) {
+          const int k = (threadIdx.x + NT * s) % HB;
+          const float cr = cr_c[s], ci = ci_c[s];
+          // packed product: bin 0 multiplies the real pair component-wise, other bins
+          // are complex products (conjugated c for grad_x)
+          const bool z = (k == 0);
+          const float a2 = z ? 0.0f : (BWDX ? ci : -ci);
+          const float a3 = z ? ci : cr;
+          const float a4 = z ? 0.0f : (BWDX ? -ci : ci);
+          const float xr = tile[rb + LayerGeo<P>::at(k)];
+          const float xi = tile[rb + LayerGeo<P>::at(bin_im_slot<P>(k))];
+          acc_r[s][t] = fmaf(cr, xr, fmaf(a2, xi, acc_r[s][t]));
+          acc_i[s][t] = fmaf(a3, xi, fmaf(a4, xr, acc_i[s][t]));
+        }
       }
     }
+    __syncthreads();
+
+    // 3. output spectra over the tile: row t*QI + ol
+  #pragma unroll
+    for (int s = 0; s < NS; ++s) {
+      const int pi = threadIdx.x + NT * s;
+      const int ol = pi / HB, k = pi % HB;
+      if (ol < QI) {
+        const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
+  #pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          // stored mirrored (slot k = Re - Im, slot p-k = Re + Im) for the Hartley-form
+          // inverse below; bin 0 keeps its real pair
+          const int rb = LayerGeo<P>::row_base(t * QI + ol);
+          tile[rb + kr] = k == 0 ? acc_r[s][t] : acc_r[s][t] - acc_i[s][t];
+          tile[rb + ki] = k == 0 ? acc_i[s][t] : acc_r[s][t] + acc_i[s][t];
+        }
+      }
+    }
+    __syncthreads();
+
   }
-  __syncthreads();
 
   // 4. rdIFFT of the TT*QI output rows straight to HBM
   ifft_rows_mirrored<P, NT, T>(tile, TT * QI, [&](int r) -> T* {
