@@ -449,6 +449,10 @@ def run_ours(args):
 
     layer["d4096_p128_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 4096, 128, 50), 1)
     layer["d4096_p512_B4096_fwd_bwd_tokens_s_per_adapter"] = round(layer_rate(4096, 4096, 512, 20), 1)
+    # block-size extremes, B = 256: one whole-row transform per block (q = 1) and q = 4
+    layer["d4096_p1024_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 4096, 1024, 50), 1)
+    layer["d4096_p4096_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 4096, 4096, 50), 1)
+    layer["d1024_p1024_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 1024, 1024, 50), 1)
 
     # LLaMA2-7B-shaped adapter stack: 32 layers x (q, v) adapters, 4096 tokens per step
     nl, B, D, p = 32, 4096, 4096, 512
