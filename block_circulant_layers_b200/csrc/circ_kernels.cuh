@@ -349,82 +349,173 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   const int nib = q / RI, njb = QJ / RJ;
   const int ngroups = HB * nib * njb;
 
-  float s_r[NG][RI][RJ], s_i[NG][RI][RJ];
-#pragma unroll
-  for (int n = 0; n < NG; ++n)
-#pragma unroll
-    for (int a = 0; a < RI; ++a)
-#pragma unroll
-      for (int b = 0; b < RJ; ++b) s_r[n][a][b] = s_i[n][a][b] = 0.0f;
+  if constexpr (RJ % 2 == 0) {
+    // S accumulators: input blocks b and b + 1 of a group on packed fp32 pairs (RJ even),
+    // the G value they share broadcast to both halves.
+    constexpr int RJP = (RJ + 1) / 2;
+    f2 s_r[NG][RI][RJP], s_i[NG][RI][RJP];
+  #pragma unroll
+    for (int n = 0; n < NG; ++n)
+  #pragma unroll
+      for (int a = 0; a < RI; ++a)
+  #pragma unroll
+        for (int b = 0; b < RJP; ++b) s_r[n][a][b] = s_i[n][a][b] = f2_bc(0.0f);
 
-  const int xrow0 = TT * q;
-  for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
-    const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
-    if (tok0 != tbeg) __syncthreads();          // previous tile fully consumed
-    // rows [0, TT*q): G; rows [TT*q, TT*q + TT*QJ): X of the CTA's blocks
-    fft_rows<P, NT, T>(tile, TT * q + TT * QJ, [&](int r) -> const T* {
-      if (r < xrow0) {
-        const int t = r / q, b = r - t * q;
-        return t < ntok ? g + (tok0 + t) * (int64_t)D + (int64_t)b * P : nullptr;
+    const int xrow0 = TT * q;
+    for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
+      const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
+      if (tok0 != tbeg) __syncthreads();          // previous tile fully consumed
+      // rows [0, TT*q): G; rows [TT*q, TT*q + TT*QJ): X of the CTA's blocks
+      fft_rows<P, NT, T>(tile, TT * q + TT * QJ, [&](int r) -> const T* {
+        if (r < xrow0) {
+          const int t = r / q, b = r - t * q;
+          return t < ntok ? g + (tok0 + t) * (int64_t)D + (int64_t)b * P : nullptr;
+        }
+        const int rr = r - xrow0;
+        const int t = rr / QJ, jl = rr - t * QJ;
+        return t < ntok ? x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
+      });
+      __syncthreads();
+  #pragma unroll
+      for (int n = 0; n < NG; ++n) {
+        const int gam = threadIdx.x + NT * n;
+        if (gam < ngroups) {
+          const int k = gam % HB;
+          const int rest = gam / HB;
+          const int ib = rest % nib, jb = rest / nib;
+          const bool z = (k == 0);
+          const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
+          for (int t = 0; t < ntok; ++t) {
+            float gr[RI], gi[RI];
+  #pragma unroll
+            for (int a = 0; a < RI; ++a) {
+              const int rb = LayerGeo<P>::row_base(t * q + ib * RI + a);
+              gr[a] = tile[rb + kr];
+              gi[a] = tile[rb + ki];
+            }
+  #pragma unroll
+            for (int bp = 0; bp < RJP; ++bp) {
+              float xr[2], xi[2];
+  #pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int b = 2 * bp + h < RJ ? 2 * bp + h : RJ - 1;   // odd RJ: the spare half repeats b
+                const int rb = LayerGeo<P>::row_base(xrow0 + t * QJ + jb * RJ + b);
+                xr[h] = tile[rb + kr];
+                xi[h] = tile[rb + ki];
+              }
+              // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)
+              const f2 vxr = f2_mk(xr[0], xr[1]);
+              const f2 vxi_re = z ? f2_bc(0.0f) : f2_mk(xi[0], xi[1]);
+              const f2 vx_im = z ? f2_mk(xi[0], xi[1]) : f2_mk(xr[0], xr[1]);
+              const f2 vxi_im = z ? f2_bc(0.0f) : f2_mk(-xi[0], -xi[1]);
+  #pragma unroll
+              for (int a = 0; a < RI; ++a) {
+                const f2 vgr = f2_bc(gr[a]), vgi = f2_bc(gi[a]);
+                s_r[n][a][bp] = f2_fma(vgr, vxr, f2_fma(vgi, vxi_re, s_r[n][a][bp]));
+                s_i[n][a][bp] = f2_fma(vgi, vx_im, f2_fma(vgr, vxi_im, s_i[n][a][bp]));
+              }
+            }
+          }
+        }
       }
-      const int rr = r - xrow0;
-      const int t = rr / QJ, jl = rr - t * QJ;
-      return t < ntok ? x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
-    });
-    __syncthreads();
-#pragma unroll
+    }
+    // add this CTA's partial packed cross-spectrum into grad_c
+  #pragma unroll
     for (int n = 0; n < NG; ++n) {
       const int gam = threadIdx.x + NT * n;
       if (gam < ngroups) {
         const int k = gam % HB;
         const int rest = gam / HB;
         const int ib = rest % nib, jb = rest / nib;
-        const bool z = (k == 0);
-        const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
-        for (int t = 0; t < ntok; ++t) {
-          float gr[RI], gi[RI];
-#pragma unroll
-          for (int a = 0; a < RI; ++a) {
-            const int rb = LayerGeo<P>::row_base(t * q + ib * RI + a);
-            gr[a] = tile[rb + kr];
-            gi[a] = tile[rb + ki];
-          }
-#pragma unroll
+        const int kim = bin_im_slot<P>(k);
+  #pragma unroll
+        for (int a = 0; a < RI; ++a)
+  #pragma unroll
           for (int b = 0; b < RJ; ++b) {
-            const int rb = LayerGeo<P>::row_base(xrow0 + t * QJ + jb * RJ + b);
-            const float xr = tile[rb + kr];
-            const float xi = tile[rb + ki];
-            // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)
-            const float xi_re = z ? 0.0f : xi;
-            const float x_im = z ? xi : xr;
-            const float xi_im = z ? 0.0f : -xi;
-#pragma unroll
+            float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
+            atomicAdd(dst + k, (b & 1) ? s_r[n][a][b / 2].y : s_r[n][a][b / 2].x);
+            atomicAdd(dst + kim, (b & 1) ? s_i[n][a][b / 2].y : s_i[n][a][b / 2].x);
+          }
+      }
+    }
+  } else {
+    float s_r[NG][RI][RJ], s_i[NG][RI][RJ];
+  #pragma unroll
+    for (int n = 0; n < NG; ++n)
+  #pragma unroll
+      for (int a = 0; a < RI; ++a)
+  #pragma unroll
+        for (int b = 0; b < RJ; ++b) s_r[n][a][b] = s_i[n][a][b] = 0.0f;
+
+    const int xrow0 = TT * q;
+    for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
+      const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
+      if (tok0 != tbeg) __syncthreads();          // previous tile fully consumed
+      // rows [0, TT*q): G; rows [TT*q, TT*q + TT*QJ): X of the CTA's blocks
+      fft_rows<P, NT, T>(tile, TT * q + TT * QJ, [&](int r) -> const T* {
+        if (r < xrow0) {
+          const int t = r / q, b = r - t * q;
+          return t < ntok ? g + (tok0 + t) * (int64_t)D + (int64_t)b * P : nullptr;
+        }
+        const int rr = r - xrow0;
+        const int t = rr / QJ, jl = rr - t * QJ;
+        return t < ntok ? x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
+      });
+      __syncthreads();
+  #pragma unroll
+      for (int n = 0; n < NG; ++n) {
+        const int gam = threadIdx.x + NT * n;
+        if (gam < ngroups) {
+          const int k = gam % HB;
+          const int rest = gam / HB;
+          const int ib = rest % nib, jb = rest / nib;
+          const bool z = (k == 0);
+          const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
+          for (int t = 0; t < ntok; ++t) {
+            float gr[RI], gi[RI];
+  #pragma unroll
             for (int a = 0; a < RI; ++a) {
-              s_r[n][a][b] = fmaf(gr[a], xr, fmaf(gi[a], xi_re, s_r[n][a][b]));
-              s_i[n][a][b] = fmaf(gi[a], x_im, fmaf(gr[a], xi_im, s_i[n][a][b]));
+              const int rb = LayerGeo<P>::row_base(t * q + ib * RI + a);
+              gr[a] = tile[rb + kr];
+              gi[a] = tile[rb + ki];
+            }
+  #pragma unroll
+            for (int b = 0; b < RJ; ++b) {
+              const int rb = LayerGeo<P>::row_base(xrow0 + t * QJ + jb * RJ + b);
+              const float xr = tile[rb + kr];
+              const float xi = tile[rb + ki];
+              // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)
+              const float xi_re = z ? 0.0f : xi;
+              const float x_im = z ? xi : xr;
+              const float xi_im = z ? 0.0f : -xi;
+  #pragma unroll
+              for (int a = 0; a < RI; ++a) {
+                s_r[n][a][b] = fmaf(gr[a], xr, fmaf(gi[a], xi_re, s_r[n][a][b]));
+                s_i[n][a][b] = fmaf(gi[a], x_im, fmaf(gr[a], xi_im, s_i[n][a][b]));
+              }
             }
           }
         }
       }
     }
-  }
-  // add this CTA's partial packed cross-spectrum into grad_c
-#pragma unroll
-  for (int n = 0; n < NG; ++n) {
-    const int gam = threadIdx.x + NT * n;
-    if (gam < ngroups) {
-      const int k = gam % HB;
-      const int rest = gam / HB;
-      const int ib = rest % nib, jb = rest / nib;
-      const int kim = bin_im_slot<P>(k);
-#pragma unroll
-      for (int a = 0; a < RI; ++a)
-#pragma unroll
-        for (int b = 0; b < RJ; ++b) {
-          float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
-          atomicAdd(dst + k, s_r[n][a][b]);
-          atomicAdd(dst + kim, s_i[n][a][b]);
-        }
+    // add this CTA's partial packed cross-spectrum into grad_c
+  #pragma unroll
+    for (int n = 0; n < NG; ++n) {
+      const int gam = threadIdx.x + NT * n;
+      if (gam < ngroups) {
+        const int k = gam % HB;
+        const int rest = gam / HB;
+        const int ib = rest % nib, jb = rest / nib;
+        const int kim = bin_im_slot<P>(k);
+  #pragma unroll
+        for (int a = 0; a < RI; ++a)
+  #pragma unroll
+          for (int b = 0; b < RJ; ++b) {
+            float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
+            atomicAdd(dst + k, s_r[n][a][b]);
+            atomicAdd(dst + kim, s_i[n][a][b]);
+          }
+      }
     }
   }
 }
