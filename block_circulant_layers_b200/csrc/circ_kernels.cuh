@@ -560,8 +560,8 @@ static cudaError_t launch_x_cfg(const void* in, const float* chat, void* out, in
 }
 
 // Launch policy (at most 32 complex accumulators per thread, NS * TT <= 32):
-//  p <= 512 : 256 threads, up to 8 output blocks per CTA (16 at p = 128), 1/2/4 tokens
-//             per CTA by B;
+//  p <= 512 : 256 threads, up to 8 output blocks per CTA (16 at p = 128 from B = 256),
+//             1/2/4 tokens per CTA by B;
 //  p >= 1024: 128 threads, one token per CTA (4 for the q = 1, p = 1024 layer; one
 //             output block per CTA for q = 1 at p >= 2048).
 template <int P, typename T, bool BWDX>
@@ -569,10 +569,13 @@ static cudaError_t launch_x_p(const void* in, const float* chat, void* out, int6
                               cudaStream_t s) {
   if constexpr (P <= 512) {
     constexpr int NT = 256;
-    // up to 8 output blocks per CTA, 16 at p = 128 (fewer CTA groups transform the same
-    // input rows; measured 7% faster at D = 4096, B = 256)
-    constexpr int NBLK = P == 128 ? 16 : 8;
-    constexpr int NS = (NBLK * (P / 2)) / NT > 0 ? (NBLK * (P / 2)) / NT : 1;
+    // up to 8 output blocks per CTA; 16 at p = 128 from B = 256 on, where fewer CTA
+    // groups transforming the same input rows pays (7% faster at D = 4096, B = 256; at
+    // B = 1 the 8-block CTAs, more of them, are 11% faster)
+    constexpr int NS = (8 * (P / 2)) / NT > 0 ? (8 * (P / 2)) / NT : 1;
+    if constexpr (P == 128) {
+      if (B >= 256) return launch_x_cfg<P, T, NT, 4, 2 * NS, BWDX>(in, chat, out, B, q, s);
+    }
     if (B >= 256 && NS * 4 <= 32) return launch_x_cfg<P, T, NT, 4, NS, BWDX>(in, chat, out, B, q, s);
     if (B >= 32) return launch_x_cfg<P, T, NT, 2, NS, BWDX>(in, chat, out, B, q, s);
     return launch_x_cfg<P, T, NT, 1, NS, BWDX>(in, chat, out, B, q, s);
