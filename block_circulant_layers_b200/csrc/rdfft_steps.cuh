@@ -78,14 +78,17 @@ struct RowTiling {
 // 16 (r / RW) bytes. So staged rows are 16-byte aligned for the bulk copies and never
 // overlap, the RW rows of a warp read disjoint banks, and consecutive warp groups are
 // shifted by one more 16-byte bank group (for the merged orbits, which one warp
-// stores for many rows at the same in-row position).
+// stores for many rows at the same in-row position). 16-bit rows of p = 256 and 512
+// take twice that SEG: with TPR*2 bytes, rows r and r + 3 (p = 512) of the merged
+// orbits' accesses fall in one bank.
 template <int P, typename T>
 struct RowSmem {
   static constexpr int ROWS = RowTiling<P>::ROWS;
   static constexpr int TPR = RowGeo<P>::TPR;
   static constexpr int RW = TPR < 32 ? 32 / TPR : 1;
   static constexpr int RAW_ROW = P * (int)sizeof(T);
-  static constexpr int SEG = TPR * (int)sizeof(T) < 16 ? 16 : TPR * (int)sizeof(T);
+  static constexpr int SEG1 = TPR * (int)sizeof(T) < 16 ? 16 : TPR * (int)sizeof(T);
+  static constexpr int SEG = (sizeof(T) == 2 && (P == 256 || P == 512)) ? 2 * SEG1 : SEG1;
   RD_HD static constexpr int raw_off(int r) { return r * (RAW_ROW + SEG) + 16 * (r / RW); }
   static constexpr int TILE_OFF = raw_off(ROWS - 1) + RAW_ROW;
   static constexpr int MBAR_OFF = TILE_OFF + ((RowGeo<P>::words(ROWS) * 4 + 15) / 16) * 16;

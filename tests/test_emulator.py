@@ -68,6 +68,22 @@ def test_bf16_forward_and_inverse(emu, p):
     assert np.all(np.abs(bf16_bits_to_f64(b) - ref_i) <= 2e-2 * np.sqrt(np.mean(ref_i ** 2)))
 
 
+@pytest.mark.parametrize("inverse", [0, 1])
+@pytest.mark.parametrize("p", [64, 128, 256, 512, 1024, 2048, 4096])
+def test_bf16_rows_equal_rounded_fp32_rows(emu, p, inverse):
+    """A bf16 row transform does the fp32 transform's arithmetic and rounds once at
+    the store: its output equals the fp32 emulation of the same input rounded to bf16
+    (nearest even), bit for bit. This pins the 16-bit store order of the staged rows
+    (odd lanes storing another element than even lanes) to the fp32 positions."""
+    rows = _rows_for(p)
+    s = sample(3500 + p + inverse, (rows, p), "bf16")
+    b = s.stored.copy()
+    f = bf16_bits_to_f64(s.stored).astype(np.float32)
+    assert emu.rdfft_emulate(b.ctypes.data, rows, p, 1, inverse) == 0
+    assert emu.rdfft_emulate(f.ctypes.data, rows, p, 0, inverse) == 0
+    assert np.array_equal(b, round_to_bf16(f.astype(np.float64)))
+
+
 def test_round_trip_and_empty(emu):
     p, rows = 1024, 3
     s = sample(4000, (rows, p), "f32")
@@ -159,7 +175,8 @@ def test_rows_kernel_shared_memory_plan(emu, p, dtype):
     """The rows kernel's shared-memory plan: staged rows 16-byte aligned (bulk copies),
     disjoint, below the tile, the tile below the mbarrier, all within the 227 KiB a CTA
     may have; the first step of pass 0 (the RW rows of a warp, TPR lanes each, reading
-    consecutive elements) conflict-free in the 32 four-byte banks from p = 128 on."""
+    consecutive elements) conflict-free in the 32 four-byte banks from p = 128 on, and
+    from p = 512 on the merged orbits' one-lane-per-row accesses too."""
     emu.rdfft_row_smem_plan.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
     out = (ctypes.c_int64 * 7000)()
     assert emu.rdfft_row_smem_plan(p, dtype, out) == 0
@@ -180,3 +197,8 @@ def test_rows_kernel_shared_memory_plan(emu, p, dtype):
                 banks.setdefault(word % 32, set()).add(word)
         worst = max(len(ws) for ws in banks.values())
         assert worst <= (2 if p == 64 else 1), (p, dtype, worst)
+    if p >= 512:
+        # the merged orbits of the last pass: one lane per row, all rows, one in-row
+        # position; the rows' staged copies start in distinct four-byte banks
+        starts = [(o // 4) % 32 for o in offs]
+        assert len(set(starts)) == rows, (p, dtype, starts)
