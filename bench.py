@@ -47,8 +47,8 @@ ROWS_KERNEL_SOURCES = ("bulk_copy.cuh", "gen_twiddles.py", "packed_fft.cuh", "rd
 
 # ncu dram bytes per launch of the dominant kernel, with the hash of the kernel
 # sources they were captured from (see profiles/); stale counters are reported null.
-TRAFFIC_CAPTURE = {"sources_sha1": "10cb0f2fa9541d68665cbe1c27f51f714c4ce95c",
-                   "bytes_per_launch": {"bf16_p4096_inv": 3453181, "bf16_p4096_fwd": 3453539}}
+TRAFFIC_CAPTURE = {"sources_sha1": "bb56009cedba847afc26dbc5d62d9596638660d6",
+                   "bytes_per_launch": {"bf16_p4096_inv": 3457606, "bf16_p4096_fwd": 3447914}}
 
 
 def kernel_sources_sha1() -> str:
@@ -448,6 +448,8 @@ def run_ours(args):
         return B / tt
 
     layer["d4096_p128_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 4096, 128, 50), 1)
+    # B = 1 (one token): latency of prepare + forward + backward
+    layer["d4096_p128_B1_fwd_bwd_us"] = round(1e6 / layer_rate(1, 4096, 128, 200), 2)
     layer["d4096_p512_B4096_fwd_bwd_tokens_s_per_adapter"] = round(layer_rate(4096, 4096, 512, 20), 1)
     # block-size extremes, B = 256: one whole-row transform per block (q = 1) and q = 4
     layer["d4096_p1024_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 4096, 1024, 50), 1)
@@ -598,6 +600,7 @@ PROFILE_CASES = {
     "circ_bwdc_d4096_p512_b4096": ("circ", (4096, 4096, 512, "bwdc")),
     "circ_fwd_d4096_p128_b256": ("circ", (256, 4096, 128, "fwd")),
     "circ_bwdc_d4096_p128_b256": ("circ", (256, 4096, 128, "bwdc")),
+    "circ_step_d4096_p128_b1": ("circ_step", (1, 4096, 128)),
 }
 
 
@@ -605,7 +608,8 @@ def run_profile_case(name: str) -> int:
     """Runs 4 launches of one kernel (the last ones are the ones to capture with ncu -s/-c).
 
     rows: a 160 MiB buffer (more than L2) of rows of p; rows_small: one 256 x 4096 tensor
-    (the bench's per-launch size); circ: the layer kernel at (B, D, p)."""
+    (the bench's per-launch size); circ: the layer kernel at (B, D, p); circ_step: the
+    layer's prepare + forward + backward at (B, D, p), every kernel of it."""
     import torch
     import block_circulant_layers_b200 as rd
     kind, a = PROFILE_CASES[name]
@@ -630,6 +634,20 @@ def run_profile_case(name: str) -> int:
         for _ in range(4):
             fn(x, p)
             undo(x, p)
+    elif kind == "circ_step":
+        B, D, p = a
+        q = D // p
+        c = torch.randn(q, q, p, device=dev, generator=gen) / D ** 0.5
+        ch = torch.empty_like(c)
+        x = torch.randn(B, D, device=dev, generator=gen).to(torch.bfloat16)
+        g = torch.randn(B, D, device=dev, generator=gen).to(torch.bfloat16)
+        y = torch.empty_like(x)
+        gx = torch.empty_like(x)
+        gc = torch.empty_like(c)
+        for _ in range(4):
+            rd.circ_prepare(c, out=ch)
+            rd.circ_fwd(x, ch, p, y=y)
+            rd.circ_bwd(g, x, ch, p, grad_x=gx, grad_c=gc)
     else:
         B, D, p, d = a
         q = D // p

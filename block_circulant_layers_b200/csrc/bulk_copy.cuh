@@ -83,7 +83,10 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, unsigned 
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 
-// Waits until this thread's committed bulk stores have completed.
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// Waits until this thread's committed bulk stores have read their shared-memory
+// sources, so the CTA may exit and its shared memory be reused. The global writes
+// finish on their own; like any write of the kernel they are visible to later work
+// in the stream once the kernel has completed.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 }  // namespace rdfft

@@ -19,7 +19,8 @@
 //  * k_circ_gc (grad_c): a persistent CTA owns a group of QJ input blocks j and a
 //    slice of the tokens; it keeps its part of the packed cross-spectrum
 //    S_ij = sum_b G_i conj(X_j) in registers across all its token tiles and adds it
-//    into grad_c once (fp32 red.add). grad_c is zeroed first and rdIFFT'd in place
+//    into grad_c once (fp32 red.add; a plain store when a single token slice covers
+//    all tokens, and grad_c then needs no zeroing). grad_c is rdIFFT'd in place
 //    after, so the output buffer is the only global storage used.
 #pragma once
 
@@ -185,18 +186,10 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
         }
       }
     };
-    load_c(0, cr_n, ci_n);
-    for (int j = 0; j < q; ++j) {                 // j: summed block (input j for fwd, output i for grad_x)
-      float cr_c[2 * NP], ci_c[2 * NP];
-  #pragma unroll
-      for (int sl = 0; sl < 2 * NP; ++sl) {
-        cr_c[sl] = cr_n[sl];
-        ci_c[sl] = ci_n[sl];
-      }
-      if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
-      // no guard on the slot here: a slot beyond the CTA's blocks has c = 0 (load_c), so
-      // its accumulators stay 0 and are never stored; slots that share a bin (all of
-      // them when NT >= p/2) share the loads of X.
+    // no guard on the slot here: a slot beyond the CTA's blocks has c = 0 (load_c), so
+    // its accumulators stay 0 and are never stored; slots that share a bin (all of
+    // them when NT >= p/2) share the loads of X.
+    auto contract = [&](int j, const float (&cr_c)[2 * NP], const float (&ci_c)[2 * NP]) {
   #pragma unroll
       for (int t = 0; t < TT; ++t) {
         const int rb = LayerGeo<P>::row_base(t * q + j);
@@ -218,6 +211,33 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
           acc_r[u][t] = f2_fma(c1, xr, f2_fma(c2, xi, acc_r[u][t]));
           acc_i[u][t] = f2_fma(c3, xi, f2_fma(c4, xr, acc_i[u][t]));
         }
+      }
+    };
+    // one token: a block's contraction is a few FMAs and cannot hide an L2 round trip,
+    // so the c_hat of KB summed blocks is requested at once (at most 32 floats), then
+    // contracted
+    constexpr int KB = TT == 1 ? (8 / NP < 8 ? 8 / NP : 8) : 1;
+    if constexpr (KB > 1) {
+      for (int j0 = 0; j0 < q; j0 += KB) {
+        float crb[KB][2 * NP], cib[KB][2 * NP];
+  #pragma unroll
+        for (int d = 0; d < KB; ++d)
+          if (j0 + d < q) load_c(j0 + d, crb[d], cib[d]);
+  #pragma unroll
+        for (int d = 0; d < KB; ++d)
+          if (j0 + d < q) contract(j0 + d, crb[d], cib[d]);
+      }
+    } else {
+      load_c(0, cr_n, ci_n);
+      for (int j = 0; j < q; ++j) {               // j: summed block (input j for fwd, output i for grad_x)
+        float cr_c[2 * NP], ci_c[2 * NP];
+  #pragma unroll
+        for (int sl = 0; sl < 2 * NP; ++sl) {
+          cr_c[sl] = cr_n[sl];
+          ci_c[sl] = ci_n[sl];
+        }
+        if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
+        contract(j, cr_c, ci_c);
       }
     }
     __syncthreads();
@@ -270,18 +290,10 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
         }
       }
     };
-    load_c(0, cr_n, ci_n);
-    for (int j = 0; j < q; ++j) {                 // j: summed block (input j for fwd, output i for grad_x)
-      float cr_c[NS], ci_c[NS];
-  #pragma unroll
-      for (int s = 0; s < NS; ++s) {
-        cr_c[s] = cr_n[s];
-        ci_c[s] = ci_n[s];
-      }
-      if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
-      // no guard on the slot here: a slot beyond the CTA's blocks has c = 0 (load_c), so
-      // its accumulators stay 0 and are never stored; without a branch, slots that share
-      // a bin (all of them when NT >= p/2) share the loads of X.
+    // no guard on the slot here: a slot beyond the CTA's blocks has c = 0 (load_c), so
+    // its accumulators stay 0 and are never stored; without a branch, slots that share
+    // a bin (all of them when NT >= p/2) share the loads of X.
+    auto contract = [&](int j, const float (&cr_c)[NS], const float (&ci_c)[NS]) {
   #pragma unroll
       for (int t = 0; t < TT; ++t) {
         const int rb = LayerGeo<P>::row_base(t * q + j);
@@ -300,6 +312,32 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
           acc_r[s][t] = fmaf(cr, xr, fmaf(a2, xi, acc_r[s][t]));
           acc_i[s][t] = fmaf(a3, xi, fmaf(a4, xr, acc_i[s][t]));
         }
+      }
+    };
+    // one token: c_hat of KB summed blocks requested at once (at most 32 floats), then
+    // contracted
+    constexpr int KB = TT == 1 ? (16 / NS < 8 ? 16 / NS : 8) : 1;
+    if constexpr (KB > 1) {
+      for (int j0 = 0; j0 < q; j0 += KB) {
+        float crb[KB][NS], cib[KB][NS];
+  #pragma unroll
+        for (int d = 0; d < KB; ++d)
+          if (j0 + d < q) load_c(j0 + d, crb[d], cib[d]);
+  #pragma unroll
+        for (int d = 0; d < KB; ++d)
+          if (j0 + d < q) contract(j0 + d, crb[d], cib[d]);
+      }
+    } else {
+      load_c(0, cr_n, ci_n);
+      for (int j = 0; j < q; ++j) {               // j: summed block (input j for fwd, output i for grad_x)
+        float cr_c[NS], ci_c[NS];
+  #pragma unroll
+        for (int s = 0; s < NS; ++s) {
+          cr_c[s] = cr_n[s];
+          ci_c[s] = ci_n[s];
+        }
+        if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
+        contract(j, cr_c, ci_c);
       }
     }
     __syncthreads();
@@ -348,6 +386,9 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   const int64_t tend = (tbeg + tok_per_cta < B) ? tbeg + tok_per_cta : B;
   const int nib = q / RI, njb = QJ / RJ;
   const int ngroups = HB * nib * njb;
+  // the only token slice: this CTA's sums are final and every (bin, i, j) of its group
+  // is one thread-group's, so it stores them instead of adding into a zeroed grad_c
+  const bool sole = (gridDim.x == 1);
 
   if constexpr (RJ % 2 == 0) {
     // S accumulators: input blocks b and b + 1 of a group on packed fp32 pairs (RJ even),
@@ -433,8 +474,15 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   #pragma unroll
           for (int b = 0; b < RJ; ++b) {
             float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
-            atomicAdd(dst + k, (b & 1) ? s_r[n][a][b / 2].y : s_r[n][a][b / 2].x);
-            atomicAdd(dst + kim, (b & 1) ? s_i[n][a][b / 2].y : s_i[n][a][b / 2].x);
+            const float vr = (b & 1) ? s_r[n][a][b / 2].y : s_r[n][a][b / 2].x;
+            const float vi = (b & 1) ? s_i[n][a][b / 2].y : s_i[n][a][b / 2].x;
+            if (sole) {
+              dst[k] = vr;
+              dst[kim] = vi;
+            } else {
+              atomicAdd(dst + k, vr);
+              atomicAdd(dst + kim, vi);
+            }
           }
       }
     }
@@ -512,8 +560,13 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   #pragma unroll
           for (int b = 0; b < RJ; ++b) {
             float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
-            atomicAdd(dst + k, s_r[n][a][b]);
-            atomicAdd(dst + kim, s_i[n][a][b]);
+            if (sole) {
+              dst[k] = s_r[n][a][b];
+              dst[kim] = s_i[n][a][b];
+            } else {
+              atomicAdd(dst + k, s_r[n][a][b]);
+              atomicAdd(dst + kim, s_i[n][a][b]);
+            }
           }
       }
     }
@@ -547,13 +600,17 @@ static cudaError_t launch_x_cfg(const void* in, const float* chat, void* out, in
                                 cudaStream_t s) {
   constexpr int QI_MAX = NS * NT / (P / 2);
   static_assert(QI_MAX >= 1, "slots must cover one block");
-  const int QI = largest_divisor_leq(q, QI_MAX);
+  const int64_t gx = (B + TT - 1) / TT;
+  if (gx > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+  int QI = largest_divisor_leq(q, QI_MAX);
+  // a handful of tokens: fewer output blocks per CTA (the spare slots idle) until the
+  // grid covers half the SMs, since every CTA waits on its own c_hat reads
+  const int half_sms = num_sms() / 2;
+  while (QI > 1 && gx * (q / QI) < half_sms) QI = largest_divisor_leq(q, QI - 1);
   const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(TT * q);
   auto kern = k_circ_x<P, T, NT, TT, NS, BWDX>;
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
-  const int64_t gx = (B + TT - 1) / TT;
-  if (gx > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   dim3 grid((unsigned)gx, (unsigned)(q / QI));
   kern<<<grid, NT, smem, s>>>(static_cast<const T*>(in), chat, static_cast<T*>(out), B, q, QI);
   return cudaGetLastError();
@@ -608,6 +665,11 @@ static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B
   if (slices > tiles) slices = (int)tiles;
   const int64_t tiles_per = (tiles + slices - 1) / slices;
   slices = (int)((tiles + tiles_per - 1) / tiles_per);
+  if (slices > 1) {
+    // several token slices add their partial sums into grad_c; one slice stores them
+    e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)q * q * P, s);
+    if (e != cudaSuccess) return e;
+  }
   dim3 grid((unsigned)slices, (unsigned)njgroups);
   kern<<<grid, NT, smem, s>>>(static_cast<const T*>(g), static_cast<const T*>(x), grad_c, B, q, QJ,
                               tiles_per * TT);
@@ -625,6 +687,11 @@ static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int6
   constexpr int HB = P / 2;
   int QJ = largest_divisor_leq(q, 8);
   while (QJ > 1 && (int64_t)HB * q * QJ > 32LL * NT) QJ = largest_divisor_leq(q, QJ - 1);
+  // a handful of token tiles: smaller input-block groups (more CTAs, each transforming
+  // all of g again) until the grid covers half the SMs
+  const int64_t ntiles = (B + TT - 1) / TT;
+  const int half_sms = num_sms() / 2;
+  while (QJ > 1 && ntiles * (q / QJ) < half_sms) QJ = largest_divisor_leq(q, QJ - 1);
   if ((int64_t)HB * q * QJ > 32LL * NT) return cudaErrorInvalidConfiguration;
   const int64_t slots = (int64_t)HB * q * QJ;                // complex accumulators per CTA
   if (q % 4 == 0 && QJ % 8 == 0 && slots <= 32LL * NT) return run_gc<P, T, NT, TT, 1, 4, 8>(g, x, grad_c, B, q, QJ, s);
@@ -647,7 +714,8 @@ static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int6
 
 // Per-p entry of the layer, instantiated once per translation unit (circ_p*.cu):
 // op 0 = forward (a = x, out = y); op 1 = grad_x (a = g, out = grad_x);
-// op 2 = grad_c accumulation (a = g, b = x, gc = grad_c, zeroed by the caller).
+// op 2 = grad_c accumulation (a = g, b = x, gc = grad_c; zeroed here when several
+// token slices add into it).
 template <int P>
 cudaError_t circ_layer_p(int op, const void* a, const void* b, const float* chat, void* out, float* gc,
                          int64_t B, int q, int dtype, cudaStream_t s) {

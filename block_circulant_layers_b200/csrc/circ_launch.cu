@@ -37,9 +37,9 @@ cudaError_t launch_circ_bwd(const void* g, const void* x, const float* c_hat, vo
   const int q = D / p;
   cudaError_t e = cudaSuccess;
   if (grad_c != nullptr) {
-    // zero, accumulate the packed cross-spectrum over all tokens, rdIFFT in place
-    e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)q * q * p, s);
-    if (e == cudaSuccess) e = circ_layer(p, 2, g, x, c_hat, nullptr, grad_c, B, q, dtype, s);
+    // the packed cross-spectrum summed over all tokens (the launcher zeroes grad_c
+    // first when several CTAs add into it), then rdIFFT in place
+    e = circ_layer(p, 2, g, x, c_hat, nullptr, grad_c, B, q, dtype, s);
     if (e == cudaSuccess) e = launch_rows(grad_c, (int64_t)q * q, p, 0, true, s);
     if (e != cudaSuccess) return e;
   }

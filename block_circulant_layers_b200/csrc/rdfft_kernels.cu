@@ -66,7 +66,7 @@ k_rows(T* __restrict__ data, int64_t rows) {
     if (threadIdx.x == 0) {
       for (int r = 0; r < nr; ++r) bulk_store(data + (row0 + r) * P, raw + SM::raw_off(r), SM::RAW_ROW);
       bulk_commit();
-      bulk_wait_all();
+      bulk_wait_read();
     }
   }
 }

@@ -135,3 +135,24 @@ def test_grad_c_overwrites_and_empty_batch(rd):
     rd.circ_bwd(e, e, c_hat, p, grad_c=gc, need_grad_x=False)
     torch.cuda.synchronize()
     assert torch.all(gc == 0)
+
+
+@pytest.mark.parametrize("B,D,p", [(1, 4096, 128), (2, 4096, 128), (1, 1024, 1024), (1, 4096, 4096),
+                                   (2, 512, 64), (3, 1536, 512)])
+def test_grad_c_single_token_slice_writes_every_element(rd, B, D, p):
+    """With so few tokens that one CTA per input-block group covers them all, grad_c is
+    stored instead of accumulated into a zeroed buffer: every element must be written
+    (grad_c starts as NaN here), and the values match the oracle."""
+    c, x, g = make_layer(B, D, p, "bf16", (520 + B, 521, 522))
+    c_hat = rd.circ_prepare(to_device(c, "f32"))
+    xd, gd = to_device(x, "bf16"), to_device(g, "bf16")
+    gc = torch.full(c_hat.shape, float("nan"), device="cuda")
+    gx = torch.empty_like(xd)
+    rd.circ_bwd(gd, xd, c_hat, p, grad_x=gx, grad_c=gc)
+    y = rd.circ_fwd(xd, c_hat, p)
+    torch.cuda.synchronize()
+    assert not torch.isnan(gc).any()
+    gx_ref, gc_ref = oracle.circ_backward(g.exact, x.exact, c.exact)
+    assert_parity(to_host_f64(gc), gc_ref, "bf16", f"grad_c B={B} D={D} p={p}")
+    assert_parity(to_host_f64(gx), gx_ref, "bf16", f"grad_x B={B} D={D} p={p}")
+    assert_parity(to_host_f64(y), oracle.circ_forward(x.exact, c.exact), "bf16", f"y B={B} D={D} p={p}")
