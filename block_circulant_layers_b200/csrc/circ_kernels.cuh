@@ -213,10 +213,9 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
         }
       }
     };
-    // one token: a block's contraction is a few FMAs and cannot hide an L2 round trip,
-    // so the c_hat of KB summed blocks is requested at once (at most 32 floats), then
-    // contracted
-    constexpr int KB = TT == 1 ? (8 / NP < 8 ? 8 / NP : 8) : 1;
+    // a block's contraction is too short to hide an L2 round trip, so the c_hat of KB
+    // summed blocks is requested at once (at most 32 floats), then contracted
+    constexpr int KB = 8 / NP < 8 ? 8 / NP : 8;
     if constexpr (KB > 1) {
       for (int j0 = 0; j0 < q; j0 += KB) {
         float crb[KB][2 * NP], cib[KB][2 * NP];
@@ -314,9 +313,10 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
         }
       }
     };
-    // one token: c_hat of KB summed blocks requested at once (at most 32 floats), then
-    // contracted
-    constexpr int KB = TT == 1 ? (16 / NS < 8 ? 16 / NS : 8) : 1;
+    // c_hat of KB summed blocks requested at once (at most 32 floats), then contracted;
+    // the 128-thread multi-token shapes (p >= 1024) are register-heavy and keep one
+    // block ahead
+    constexpr int KB = (P <= 512 || TT == 1) ? (16 / NS < 8 ? 16 / NS : 8) : 1;
     if constexpr (KB > 1) {
       for (int j0 = 0; j0 < q; j0 += KB) {
         float crb[KB][NS], cib[KB][NS];
