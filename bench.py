@@ -47,8 +47,8 @@ ROWS_KERNEL_SOURCES = ("bulk_copy.cuh", "gen_twiddles.py", "packed_fft.cuh", "rd
 
 # ncu dram bytes per launch of the dominant kernel, with the hash of the kernel
 # sources they were captured from (see profiles/); stale counters are reported null.
-TRAFFIC_CAPTURE = {"sources_sha1": "bb56009cedba847afc26dbc5d62d9596638660d6",
-                   "bytes_per_launch": {"bf16_p4096_inv": 3457606, "bf16_p4096_fwd": 3447914}}
+TRAFFIC_CAPTURE = {"sources_sha1": "f012d5231f58743da7fa29046234bcb9e2073c77",
+                   "bytes_per_launch": {"bf16_p4096_inv": 3443344, "bf16_p4096_fwd": 3410886}}
 
 
 def kernel_sources_sha1() -> str:
@@ -589,6 +589,8 @@ PROFILE_CASES = {
     # name: (kind, args) -- one kernel on a buffer larger than L2, for ncu captures
     "rdfft_bf16_512_fwd": ("rows", (512, "bf16", "fwd")),
     "rdfft_bf16_512_inv": ("rows", (512, "bf16", "inv")),
+    "rdfft_bf16_1024_fwd": ("rows", (1024, "bf16", "fwd")),
+    "rdfft_bf16_2048_fwd": ("rows", (2048, "bf16", "fwd")),
     "rdfft_bf16_4096_fwd": ("rows", (4096, "bf16", "fwd")),
     "rdfft_bf16_4096_inv": ("rows", (4096, "bf16", "inv")),
     "rdfft_f32_4096_fwd": ("rows", (4096, "f32", "fwd")),

@@ -267,6 +267,25 @@ int rdfft_row_smem_plan(int p, int dtype, int64_t* out) {
 #undef RD_PCASE
 }
 
+// Tile geometry of the rows kernel for row length p: out[0] = S (one pad word per 2^S
+// elements), out[1] = rows per CTA, out[2 + r] = word offset of tile row r.
+int rdfft_row_tile_plan(int p, int64_t* out) {
+#define RD_TCASE(PP)                                                                   \
+  case PP: {                                                                           \
+    using G = rdfft::RowGeo<PP>;                                                       \
+    constexpr int R = rdfft::RowTiling<PP>::ROWS;                                      \
+    out[0] = G::S;                                                                     \
+    out[1] = R;                                                                        \
+    for (int r = 0; r < R; ++r) out[2 + r] = G::row_base(r);                           \
+    return 0;                                                                          \
+  }
+  switch (p) {
+    RD_TCASE(64) RD_TCASE(128) RD_TCASE(256) RD_TCASE(512) RD_TCASE(1024) RD_TCASE(2048) RD_TCASE(4096)
+    default: return 1;
+  }
+#undef RD_TCASE
+}
+
 // Positions of the first n elements of the generic orbit with residue r of a pass
 // that starts at block size H (the kernels' orbit_pos), for the index-model test.
 void rdfft_orbit_positions(int H, int r, int n, int* out) {

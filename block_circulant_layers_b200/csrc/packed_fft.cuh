@@ -415,7 +415,7 @@ RD_HD void orbit_stages(float (&a)[E], int r) {
 // scatter and orbit gather/scatter fall in distinct banks (checked by a bank model),
 // and because every row/block base is a multiple of 2^S, each access is a per-thread
 // base register plus a compile-time offset.
-template <int P_, int EPT_>
+template <int P_, int EPT_, int SKEW_ = 0>
 struct Geo {
   static constexpr int P = P_;
   static_assert(P >= 2 && P <= kMaxP && (P & (P - 1)) == 0, "p must be a power of two in [2, 4096]");
@@ -433,16 +433,22 @@ struct Geo {
   // Row r starts at r * RS plus one extra word per RW rows, RW being the rows that
   // share a warp (32 / TPR, or 1): rows of one warp keep the bank pattern above, and
   // the 32 rows whose merged orbits one warp processes get 32 distinct bank offsets.
+  // When a warp never spans two rows (RW = 1), row r is shifted by SKEW_ * r words
+  // instead; that moves no access of a warp relative to another, only the merged
+  // orbits of different rows, which one warp processes together.
   static constexpr int RS = P + (P >> S);
   static constexpr int RW = TPR < 32 ? 32 / TPR : 1;
-  RD_HD static constexpr int row_base(int r) { return r * RS + (RW > 1 ? r / RW : 0); }
+  RD_HD static constexpr int row_base(int r) { return r * RS + (RW > 1 ? r / RW : SKEW_ * r); }
   // words of a tile of `rows` rows (plus one spare word)
   RD_HD static constexpr int words(int rows) { return row_base(rows) + 1; }
 };
 
-// The geometry of the standalone transforms: two passes for every p >= 64.
+// The geometry of the standalone transforms. Rows of p >= 1024 (one warp or more per
+// row) are skewed by 4 words: the merged orbits of pass 1, one per (row, block), then
+// fall in distinct banks (at p = 1024 they were 4-way conflicts, 18% of the kernel's
+// shared-memory wavefronts in a bank model of all its accesses).
 template <int P>
-using RowGeo = Geo<P, ept_for(P)>;
+using RowGeo = Geo<P, ept_for(P), 4>;
 
 template <class G, int K>
 struct PassShape {

@@ -84,6 +84,28 @@ def test_bf16_rows_equal_rounded_fp32_rows(emu, p, inverse):
     assert np.array_equal(b, round_to_bf16(f.astype(np.float64)))
 
 
+@pytest.mark.parametrize("p", [512, 1024, 2048, 4096])
+def test_rows_kernel_merged_orbits_spread_over_banks(emu, p):
+    """The merged orbits of an orbit pass are run one per thread by the first threads of
+    the CTA, one (row, block) each, all at the same in-block position: the rows kernel's
+    tile layout must put them in distinct four-byte banks, in every pass."""
+    emu.rdfft_row_tile_plan.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
+    out = (ctypes.c_int64 * 64)()
+    assert emu.rdfft_row_tile_plan(p, out) == 0
+    S, rows = int(out[0]), int(out[1])
+    bases = [int(out[2 + r]) for r in range(rows)]
+    s0 = (ctypes.c_int * 8)()
+    s1 = (ctypes.c_int * 8)()
+    npass = emu.rdfft_plan(p, s0, s1)
+    at = lambda n: n + (n >> S)
+    for k in range(1, npass):
+        H, LB = 1 << s0[k], 1 << s1[k]
+        nb, hh, n = p // LB, H // 2, 2 * LB // H
+        for l in range(n):
+            banks = [(b + at(beta * LB + l * hh)) % 32 for b in bases for beta in range(nb)]
+            assert len(set(banks)) == len(banks), (p, k, l, banks)
+
+
 def test_round_trip_and_empty(emu):
     p, rows = 1024, 3
     s = sample(4000, (rows, p), "f32")
