@@ -31,10 +31,9 @@
 
 namespace rdfft {
 
-// The layer kernels transform rows with 32 elements per thread (three passes at
-// p >= 1024): their registers are shared with the contraction's accumulators.
-template <int P>
-using LayerGeo = Geo<P, kEPT>;
+// The layer kernels' tiles use LayerGeo (packed_fft.cuh): 32 elements per thread,
+// three passes at p >= 1024, since their registers are shared with the contraction's
+// accumulators.
 
 // ------------------------------------------------------------- tile row passes
 // Orbit pass K (tile -> tile) over tile rows [0, NR): every thread runs the generic

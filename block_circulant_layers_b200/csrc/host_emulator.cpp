@@ -72,7 +72,7 @@ void emu_rows(T* data, int64_t rows, int ept) {
       emu_geo<RowGeo<P>, RowTiling<P>::ROWS, INV, T>(data, rows);
     } else {
       // the layer kernels' geometry: 32 elements per thread, rows of a 128-thread CTA
-      using G = Geo<P, kEPT>;
+      using G = LayerGeo<P>;
       emu_geo<G, (128 / G::TPR > 0 ? 128 / G::TPR : 1), INV, T>(data, rows);
     }
   }
@@ -83,7 +83,7 @@ void emu_rows(T* data, int64_t rows, int ept) {
 // pass to global with the mirror epilogue. ROWS rows per emulated CTA.
 template <int P, typename T>
 void emu_hartley_inverse(T* data, int64_t rows) {
-  using G = Geo<P, kEPT>;
+  using G = LayerGeo<P>;
   constexpr int TPR = G::TPR;
   constexpr int ROWS = 128 / TPR > 0 ? 128 / TPR : 1;
   std::vector<float> tile(G::words(ROWS), 0.0f);
@@ -284,6 +284,23 @@ int rdfft_row_tile_plan(int p, int64_t* out) {
     default: return 1;
   }
 #undef RD_TCASE
+}
+
+// Tile geometry of the layer kernels for row length p: out[0] = S, out[1 + r] = word
+// offset of tile row r for r < rows.
+int rdfft_layer_tile_plan(int p, int rows, int64_t* out) {
+#define RD_LCASE(PP)                                                                   \
+  case PP: {                                                                           \
+    using G = rdfft::LayerGeo<PP>;                                                     \
+    out[0] = G::S;                                                                     \
+    for (int r = 0; r < rows; ++r) out[1 + r] = G::row_base(r);                        \
+    return 0;                                                                          \
+  }
+  switch (p) {
+    RD_LCASE(64) RD_LCASE(128) RD_LCASE(256) RD_LCASE(512) RD_LCASE(1024) RD_LCASE(2048) RD_LCASE(4096)
+    default: return 1;
+  }
+#undef RD_LCASE
 }
 
 // Positions of the first n elements of the generic orbit with residue r of a pass

@@ -450,6 +450,12 @@ struct Geo {
 template <int P>
 using RowGeo = Geo<P, ept_for(P), 4>;
 
+// The geometry of the layer kernels' tiles: 32 elements per thread. Their tiles hold up
+// to 16 rows at p >= 1024 (grad_c), so rows are skewed by one word: one warp's merged
+// orbits, (row, block) pairs, then cover 32 distinct banks.
+template <int P>
+using LayerGeo = Geo<P, kEPT, 1>;
+
 template <class G, int K>
 struct PassShape {
   static constexpr int H = 1 << G::s0(K);

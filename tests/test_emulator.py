@@ -106,6 +106,31 @@ def test_rows_kernel_merged_orbits_spread_over_banks(emu, p):
             assert len(set(banks)) == len(banks), (p, k, l, banks)
 
 
+@pytest.mark.parametrize("p", [1024, 2048, 4096])
+def test_layer_tile_merged_orbits_spread_over_banks(emu, p):
+    """The layer kernels run the merged orbits of up to 16 tile rows (grad_c at p = 1024)
+    one per thread, consecutive threads taking consecutive (row, block) pairs: every warp
+    of them must fall in distinct four-byte banks, in every pass."""
+    rows = 16
+    emu.rdfft_layer_tile_plan.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int64)]
+    out = (ctypes.c_int64 * 64)()
+    assert emu.rdfft_layer_tile_plan(p, rows, out) == 0
+    S = int(out[0])
+    bases = [int(out[1 + r]) for r in range(rows)]
+    s0 = (ctypes.c_int * 8)()
+    s1 = (ctypes.c_int * 8)()
+    npass = emu.rdfft_plan(p, s0, s1)        # the layer's pass plan (32 elements per thread)
+    at = lambda n: n + (n >> S)
+    for k in range(1, npass):
+        H, LB = 1 << s0[k], 1 << s1[k]
+        nb, hh, n = p // LB, H // 2, 2 * LB // H
+        mus = list(range(rows * nb))
+        for w in range(0, len(mus), 32):
+            for l in range(n):
+                banks = [(bases[mu // nb] + at((mu % nb) * LB + l * hh)) % 32 for mu in mus[w:w + 32]]
+                assert len(set(banks)) == len(banks), (p, k, l, banks)
+
+
 def test_round_trip_and_empty(emu):
     p, rows = 1024, 3
     s = sample(4000, (rows, p), "f32")
