@@ -371,8 +371,8 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
 
 // ---------------------------------------------------------------------- grad_c
 // Thread group gamma = (k, ib, jb): bin k, output blocks i = ib*RI .. +RI, input
-// blocks jl = jb*RJ .. +RJ of the CTA's QJ-block group. The tile holds, per token
-// tile, G for rows t*q + i and X for rows TT*q + t*QJ + jl.
+// blocks jl = jb*RJ .. +RJ of the CTA's QJ-block group. The tile holds, per tile of
+// ntok <= TT tokens, G for rows t*q + i and X for rows ntok*q + t*QJ + jl.
 template <int P, typename T, int NT, int TT, int NG, int RI, int RJ>
 __global__ void __launch_bounds__(NT, 1)
 k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ grad_c,
@@ -401,19 +401,20 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   #pragma unroll
         for (int b = 0; b < RJP; ++b) s_r[n][a][b] = s_i[n][a][b] = f2_bc(0.0f);
 
-    const int xrow0 = TT * q;
     for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
       const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
       if (tok0 != tbeg) __syncthreads();          // previous tile fully consumed
-      // rows [0, TT*q): G; rows [TT*q, TT*q + TT*QJ): X of the CTA's blocks
-      fft_rows<P, NT, T>(tile, TT * q + TT * QJ, [&](int r) -> const T* {
+      // rows [0, ntok*q): G; rows [ntok*q, ntok*(q + QJ)): X of the CTA's blocks. A
+      // partial tile (a ragged tail, a handful of tokens) transforms only its rows.
+      const int xrow0 = ntok * q;
+      fft_rows<P, NT, T>(tile, ntok * (q + QJ), [&](int r) -> const T* {
         if (r < xrow0) {
           const int t = r / q, b = r - t * q;
-          return t < ntok ? g + (tok0 + t) * (int64_t)D + (int64_t)b * P : nullptr;
+          return g + (tok0 + t) * (int64_t)D + (int64_t)b * P;
         }
         const int rr = r - xrow0;
         const int t = rr / QJ, jl = rr - t * QJ;
-        return t < ntok ? x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
+        return x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P;
       });
       __syncthreads();
   #pragma unroll
@@ -494,19 +495,20 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   #pragma unroll
         for (int b = 0; b < RJ; ++b) s_r[n][a][b] = s_i[n][a][b] = 0.0f;
 
-    const int xrow0 = TT * q;
     for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
       const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
       if (tok0 != tbeg) __syncthreads();          // previous tile fully consumed
-      // rows [0, TT*q): G; rows [TT*q, TT*q + TT*QJ): X of the CTA's blocks
-      fft_rows<P, NT, T>(tile, TT * q + TT * QJ, [&](int r) -> const T* {
+      // rows [0, ntok*q): G; rows [ntok*q, ntok*(q + QJ)): X of the CTA's blocks. A
+      // partial tile (a ragged tail, a handful of tokens) transforms only its rows.
+      const int xrow0 = ntok * q;
+      fft_rows<P, NT, T>(tile, ntok * (q + QJ), [&](int r) -> const T* {
         if (r < xrow0) {
           const int t = r / q, b = r - t * q;
-          return t < ntok ? g + (tok0 + t) * (int64_t)D + (int64_t)b * P : nullptr;
+          return g + (tok0 + t) * (int64_t)D + (int64_t)b * P;
         }
         const int rr = r - xrow0;
         const int t = rr / QJ, jl = rr - t * QJ;
-        return t < ntok ? x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
+        return x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P;
       });
       __syncthreads();
   #pragma unroll
@@ -682,7 +684,7 @@ template <int P, typename T>
 static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int64_t B, int q,
                                cudaStream_t s) {
   constexpr int NT = 512;
-  constexpr int TT = (P >= 2048) ? 1 : 2;
+  constexpr int TT = (P >= 2048) ? 1 : (P >= 1024 ? 2 : 4);
   constexpr int HB = P / 2;
   int QJ = largest_divisor_leq(q, 8);
   while (QJ > 1 && (int64_t)HB * q * QJ > 32LL * NT) QJ = largest_divisor_leq(q, QJ - 1);
