@@ -27,6 +27,7 @@
 #include <cuda_runtime.h>
 
 #include "internal.h"
+#include "layer_policy.h"
 #include "packed_fft.cuh"
 
 namespace rdfft {
@@ -588,12 +589,6 @@ static cudaError_t set_smem(KernelT kernel, size_t bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
 }
 
-static int largest_divisor_leq(int q, int cap) {
-  for (int d = cap; d >= 1; --d)
-    if (q % d == 0) return d;
-  return 1;
-}
-
 // Forward / grad_x: NT threads, TT tokens per CTA, NS bins per thread, so a CTA
 // covers up to NS*NT/(P/2) output blocks.
 template <int P, typename T, int NT, int TT, int NS, bool BWDX>
@@ -603,11 +598,7 @@ static cudaError_t launch_x_cfg(const void* in, const float* chat, void* out, in
   static_assert(QI_MAX >= 1, "slots must cover one block");
   const int64_t gx = (B + TT - 1) / TT;
   if (gx > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  int QI = largest_divisor_leq(q, QI_MAX);
-  // a handful of tokens: fewer output blocks per CTA (the spare slots idle) until the
-  // grid covers half the SMs, since every CTA waits on its own c_hat reads
-  const int half_sms = num_sms() / 2;
-  while (QI > 1 && gx * (q / QI) < half_sms) QI = largest_divisor_leq(q, QI - 1);
+  const int QI = layer_qi(q, QI_MAX, gx, num_sms());
   const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(TT * q);
   auto kern = k_circ_x<P, T, NT, TT, NS, BWDX>;
   cudaError_t e = set_smem(kern, smem);
@@ -661,11 +652,8 @@ static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
   const int njgroups = q / QJ;
-  int slices = (num_sms() + njgroups - 1) / njgroups;
-  const int64_t tiles = (B + TT - 1) / TT;
-  if (slices > tiles) slices = (int)tiles;
-  const int64_t tiles_per = (tiles + slices - 1) / slices;
-  slices = (int)((tiles + tiles_per - 1) / tiles_per);
+  int64_t tiles_per = 1;
+  const int slices = layer_gc_slices(njgroups, (B + TT - 1) / TT, num_sms(), &tiles_per);
   if (slices > 1) {
     // several token slices add their partial sums into grad_c; one slice stores them
     e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)q * q * P, s);
@@ -686,13 +674,7 @@ static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int6
   constexpr int NT = 512;
   constexpr int TT = (P >= 2048) ? 1 : (P >= 1024 ? 2 : 4);
   constexpr int HB = P / 2;
-  int QJ = largest_divisor_leq(q, 8);
-  while (QJ > 1 && (int64_t)HB * q * QJ > 32LL * NT) QJ = largest_divisor_leq(q, QJ - 1);
-  // a handful of token tiles: smaller input-block groups (more CTAs, each transforming
-  // all of g again) until the grid covers half the SMs
-  const int64_t ntiles = (B + TT - 1) / TT;
-  const int half_sms = num_sms() / 2;
-  while (QJ > 1 && ntiles * (q / QJ) < half_sms) QJ = largest_divisor_leq(q, QJ - 1);
+  const int QJ = layer_qj(q, HB, 32LL * NT, (B + TT - 1) / TT, num_sms());
   if ((int64_t)HB * q * QJ > 32LL * NT) return cudaErrorInvalidConfiguration;
   const int64_t slots = (int64_t)HB * q * QJ;                // complex accumulators per CTA
   if (q % 4 == 0 && QJ % 8 == 0 && slots <= 32LL * NT) return run_gc<P, T, NT, TT, 1, 4, 8>(g, x, grad_c, B, q, QJ, s);

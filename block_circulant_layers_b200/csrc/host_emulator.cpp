@@ -9,6 +9,7 @@
 
 #include <vector>
 
+#include "layer_policy.h"
 #include "rdfft2d_steps.cuh"
 #include "rdfft_steps.cuh"
 
@@ -301,6 +302,15 @@ int rdfft_layer_tile_plan(int p, int rows, int64_t* out) {
     default: return 1;
   }
 #undef RD_LCASE
+}
+
+// The layer launchers' shape rules (layer_policy.h), for the CPU tests.
+int rdfft_layer_qi(int q, int qi_max, int64_t gx, int n_sm) { return rdfft::layer_qi(q, qi_max, gx, n_sm); }
+int rdfft_layer_qj(int q, int hb, int64_t max_slots, int64_t ntiles, int n_sm) {
+  return rdfft::layer_qj(q, hb, max_slots, ntiles, n_sm);
+}
+int rdfft_layer_gc_slices(int njgroups, int64_t ntiles, int n_sm, int64_t* tiles_per) {
+  return rdfft::layer_gc_slices(njgroups, ntiles, n_sm, tiles_per);
 }
 
 // Positions of the first n elements of the generic orbit with residue r of a pass

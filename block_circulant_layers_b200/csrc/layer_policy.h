@@ -1,0 +1,50 @@
+// Launch-shape rules of the block-circulant layer kernels. Plain host arithmetic,
+// shared by the CUDA launchers (circ_kernels.cuh) and the host test library, so the
+// rules are checked on the CPU.
+#pragma once
+
+#include <stdint.h>
+
+namespace rdfft {
+
+// Largest divisor of q that is at most cap (at least 1).
+inline int largest_divisor_leq(int q, int cap) {
+  for (int d = cap; d >= 1; --d)
+    if (q % d == 0) return d;
+  return 1;
+}
+
+// Output blocks per CTA of the forward / grad_x kernel: as many as the CTA's slots
+// cover (qi_max, a divisor of q), and fewer while the grid of gx token groups times
+// q / QI block groups would cover fewer than half of the n_sm SMs. The spare slots of
+// a CTA then idle; every CTA waits on its own c_hat reads, so more CTAs finish sooner.
+inline int layer_qi(int q, int qi_max, int64_t gx, int n_sm) {
+  int qi = largest_divisor_leq(q, qi_max);
+  while (qi > 1 && gx * (q / qi) < n_sm / 2) qi = largest_divisor_leq(q, qi - 1);
+  return qi;
+}
+
+// Input blocks per grad_c CTA group: a divisor of q, at most 8, with at most
+// max_slots complex accumulators per CTA (hb bins x q output blocks x QJ), and fewer
+// while ntiles token tiles times q / QJ groups would cover fewer than half the SMs
+// (each group then transforms all of g again, which only pays with few tokens).
+inline int layer_qj(int q, int hb, int64_t max_slots, int64_t ntiles, int n_sm) {
+  int qj = largest_divisor_leq(q, 8);
+  while (qj > 1 && (int64_t)hb * q * qj > max_slots) qj = largest_divisor_leq(q, qj - 1);
+  while (qj > 1 && ntiles * (q / qj) < n_sm / 2) qj = largest_divisor_leq(q, qj - 1);
+  return qj;
+}
+
+// Token slices of the persistent grad_c grid: about n_sm CTAs over the njgroups
+// input-block groups, each slice a whole number of token tiles (*tiles_per, at least
+// 1). Returns the number of slices (at least 1).
+inline int layer_gc_slices(int njgroups, int64_t ntiles, int n_sm, int64_t* tiles_per) {
+  if (ntiles < 1) ntiles = 1;
+  int64_t slices = (n_sm + njgroups - 1) / njgroups;
+  if (slices < 1) slices = 1;
+  if (slices > ntiles) slices = ntiles;
+  *tiles_per = (ntiles + slices - 1) / slices;
+  return (int)((ntiles + *tiles_per - 1) / *tiles_per);
+}
+
+}  // namespace rdfft
