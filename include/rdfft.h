@@ -171,11 +171,13 @@ int circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p
  *            g, x, c_hat or grad_c (RDFFT_EOVERLAP).
  *   grad_c : q x q x p fp32 in the spatial domain (same layout as c), overwritten
  *            with the gradient summed over all B tokens; may be NULL to skip it.
- *            The buffer is used in place: it is zeroed, accumulates the packed
- *            cross-spectrum, and ends with an in-place rdIFFT of its q*q rows.
- *            Must not overlap g, x or c_hat (RDFFT_EOVERLAP).
- * The grad_c sum over tokens is accumulated with fp32 atomic adds, so its last bits
- * may differ between runs; grad_x and the forward are deterministic.
+ *            The buffer is used in place: it receives the packed cross-spectrum and
+ *            ends with an in-place rdIFFT of its q*q rows. Its prior contents never
+ *            matter. Must not overlap g, x or c_hat (RDFFT_EOVERLAP).
+ * When the tokens are split over several CTAs, the grad_c sum over tokens is
+ * accumulated with fp32 atomic adds into a zeroed buffer, so its last bits may differ
+ * between runs. With a handful of tokens one CTA per block group sums them all and
+ * stores the result, and grad_c is deterministic; grad_x and the forward always are.
  */
 int circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
              int64_t B, int D, int p, int dtype, rdfft_stream_t stream);
