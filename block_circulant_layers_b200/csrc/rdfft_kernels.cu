@@ -31,9 +31,11 @@ template <int P, bool INV, typename T>
 __global__ void __launch_bounds__(RowTiling<P>::THREADS)
 k_rows(T* __restrict__ data, int64_t rows) {
   constexpr int ROWS = RowTiling<P>::ROWS;
+  griddep_wait();                                     // earlier work on these rows is done
   if constexpr (P <= 32) {
     const int64_t row = (int64_t)blockIdx.x * ROWS + threadIdx.x;
     if (row < rows) row_small<P, INV, T>(data + row * P);
+    griddep_launch_dependents();
   } else {
     using G = RowGeo<P>;
     using SM = RowSmem<P, T>;
@@ -63,6 +65,7 @@ k_rows(T* __restrict__ data, int64_t rows) {
     run_steps<G, INV, 0, ROWS, T>(tile, lrow, v, rowptr, rowok);
     fence_smem_to_async();
     __syncthreads();
+    griddep_launch_dependents();                      // the next launch may be scheduled
     if (threadIdx.x == 0) {
       for (int r = 0; r < nr; ++r) bulk_store(data + (row0 + r) * P, raw + SM::raw_off(r), SM::RAW_ROW);
       bulk_commit();
@@ -106,8 +109,19 @@ static cudaError_t launch_pi(T* d, int64_t rows, cudaStream_t s) {
       if (e != cudaSuccess) return e;
     }
   }
-  k_rows<P, INV, T><<<(unsigned)grid, RowTiling<P>::THREADS, smem, s>>>(d, rows);
-  return cudaGetLastError();
+  // programmatic stream serialization: the next rows launch in the stream can be
+  // scheduled while this one drains; each CTA waits (griddep_wait) before touching data
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(RowTiling<P>::THREADS);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k_rows<P, INV, T>, d, rows);
 }
 
 template <int P, typename T>
