@@ -3,28 +3,40 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
-Workload (one 256 x 4096 tensor of N(0,1) reals viewed as rows of p = 512 and of
-p = 4096, bf16, in-place forward rdFFT then rdIFFT). One STEP transforms a pool of
-POOL distinct such tensors in each view (forward then inverse, in place), issued
-round-robin on STREAMS CUDA streams and replayed as one CUDA graph; the pool holds
-256 MiB, twice the L2, so every launch reads HBM. The metric is whole-job GB/s:
-algorithmic bytes (one read and one write of every element per transform) over the
-device time of K steps, max over ranks. Rank r of N transforms its own pool (weak
-scaling, no collective on the data path).
+Workload: one 256 x 4096 tensor of N(0,1) reals viewed as rows of p = 512 and of
+p = 4096, bf16, transformed in place by rdFFT and then rdIFFT. The bench keeps a
+pool of POOL distinct such tensors per view (256 MiB per view, twice the L2). One
+ROUND is four sweeps over the pools: the forward of every p = 512 tensor, the
+forward of every p = 4096 tensor, then the two inverses. Every tensor is therefore
+last touched 768 MiB of traffic before its next transform, so every launch reads
+HBM, and each tensor returns to its original values once a round. A sweep issues
+its POOL launches round-robin on STREAMS CUDA streams and is replayed as one CUDA
+graph. One STEP is R rounds, R fixed after warm-up so that a step takes about
+STEP_TARGET_S seconds (so the clock sampler sees the timed region). The metric is
+whole-job GB/s: algorithmic bytes (one read and one write of every element per
+transform) over the device time of K steps, max over ranks. Rank r of N transforms
+its own pools (weak scaling, no collective on the data path).
 
-The same JSON line carries: a per-kernel breakdown, the roofline of the dominant
-kernel, an end-to-end figure through the public API with pinned host buffers, the
-block-circulant layer's tokens/s at D = 4096 (bf16), SM clocks sampled during the
-timed region, and the float64 CPU oracle timed on a bounded sample (rank 0, N = 1).
+The timed region records a CUDA event before every sweep, so the per-kernel
+breakdown and the roofline of the dominant kernel come from the same timed launches
+as the headline. The JSON line also carries one large launch per kernel (the
+asymptotic GB/s), an end-to-end figure through the public API with pinned host
+buffers, the block-circulant layer at the D = 4096 workloads (tokens/s forward,
+backward and both, GB/s, %HBM and %FP32 per kernel, and the float64 oracle timed on
+the host beside it), SM clocks sampled during the timed region, and the float64 CPU
+oracle timed on the rdFFT workload (rank 0, N = 1).
 
 --impl reference times the float64 CPU oracle on the host cores instead (rank 0
-only), on a bounded slice of the same workload per step.
+only): each step is one whole 256 x 4096 tensor in each view, forward and inverse,
+the same sample the cpu_baseline of our arm uses.
 """
 from __future__ import annotations
 
 import argparse
+import contextlib
 import hashlib
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -39,9 +51,13 @@ if ROOT not in sys.path:
 METRIC = "rdFFT fwd/inv GB/s (% HBM peak); circulant layer tokens/s, D=4096 bf16"
 PS = (512, 4096)
 ELEMS = 256 * 4096          # reals per tensor
-POOL = 64                   # tensors per view; 2 MiB each in bf16
+POOL = 128                  # tensors per view; 2 MiB each in bf16, 256 MiB per view
 STREAMS = 8
+SWEEPS = (("fwd", 512), ("fwd", 4096), ("inv", 512), ("inv", 4096))
+STEP_TARGET_S = 0.06
 FALLBACK_HBM_GBS = 6650.0
+FP32_LANES_PER_SM = 128     # FP32 FMA lanes per B200 SM (4 sub-partitions x 32)
+NOMINAL_SM_MHZ = 1965.0
 
 ROWS_KERNEL_SOURCES = ("bulk_copy.cuh", "gen_twiddles.py", "packed_fft.cuh", "rdfft_kernels.cu", "rdfft_steps.cuh")
 
@@ -72,9 +88,20 @@ def measured_peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+@contextlib.contextmanager
+def nvtx(name: str):
+    """NVTX range around a phase of the bench (visible in nsys / ncu range filters)."""
+    import torch
+    torch.cuda.nvtx.range_push(name)
+    try:
+        yield
+    finally:
+        torch.cuda.nvtx.range_pop()
+
+
 # ----------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi clocks / throttle reasons sampled every 100 ms while running."""
+    """nvidia-smi clocks / throttle reasons sampled every 50 ms while running."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -87,7 +114,7 @@ class ClockSampler:
         self.thread = None
 
     def __enter__(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
         if self.uuid:
             cmd[1:1] = ["-i", self.uuid]
         try:
@@ -97,6 +124,12 @@ class ClockSampler:
         except Exception:
             self.proc = None
         return self
+
+    def wait_first(self, timeout: float = 5.0):
+        """Blocks until the first sample has arrived (nvidia-smi takes a moment to start)."""
+        t0 = time.time()
+        while self.proc is not None and not self.lines and time.time() - t0 < timeout:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -115,7 +148,7 @@ class ClockSampler:
     def summary(self, t0: float, t1: float):
         sm, mx, reasons = [], [], set()
         for ts, line in self.lines:
-            if not (t0 <= ts <= t1 + 0.15):
+            if not (t0 <= ts <= t1 + 0.05):
                 continue
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
@@ -150,6 +183,13 @@ def max_over_ranks(x: float, world: int, device) -> float:
 def rank_seed(rank: int) -> int:
     """Seed of a rank's pool: every rank transforms its own distinct data."""
     return 1000 + rank
+
+
+def rounds_per_step(t_round: float, target: float = STEP_TARGET_S) -> int:
+    """Rounds in one step so that a step takes about `target` seconds (at least 1)."""
+    if not (t_round > 0):
+        return 1
+    return max(1, int(math.ceil(target / t_round)))
 
 
 def graph_of(fn, torch):
@@ -191,6 +231,12 @@ def fanout(fn_per_item, items, nstreams, torch):
         cur.wait_stream(st)
 
 
+def fp32_peak_tflops(sm_mhz: float | None, n_sm: int) -> float:
+    """Nominal FP32 CUDA-core peak: SMs x FP32 lanes x 2 flop (one FMA) x SM clock."""
+    mhz = sm_mhz if sm_mhz else NOMINAL_SM_MHZ
+    return n_sm * FP32_LANES_PER_SM * 2 * mhz * 1e6 / 1e12
+
+
 # ---------------------------------------------------------------- oracle (CPU)
 def cpu_threads():
     try:
@@ -203,8 +249,21 @@ def cpu_threads():
     return len(os.sched_getaffinity(0))
 
 
-def oracle_slice(rows512: int, rows4096: int, seed: int = 2):
-    """Oracle forward + inverse on a slice of the workload; returns (bytes, seconds).
+@contextlib.contextmanager
+def one_core():
+    """Limits the oracle's BLAS to one thread inside the block."""
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        yield False
+        return
+    with threadpool_limits(limits=1, user_api="blas"):
+        yield True
+
+
+def oracle_tensor(seed: int):
+    """Oracle forward + inverse of one whole 256 x 4096 tensor in each view (2048 rows
+    of p = 512, 256 rows of p = 4096); returns (bytes, seconds).
 
     Bytes count like the GPU metric: bf16 storage, one read and one write of every
     element per transform."""
@@ -212,16 +271,43 @@ def oracle_slice(rows512: int, rows4096: int, seed: int = 2):
     from synthetic import sample
     nbytes = 0
     t = 0.0
-    for p, rows in ((512, rows512), (4096, rows4096)):
-        if rows <= 0:
-            continue
-        s = sample(seed, (rows, p), "bf16")
+    for p in PS:
+        s = sample(seed, (ELEMS // p, p), "bf16")
         t0 = time.perf_counter()
         y = oracle.dft_packed(s.exact)
         oracle.idft_packed(y)
         t += time.perf_counter() - t0
-        nbytes += 2 * 2 * rows * p * 2
+        nbytes += 2 * 2 * ELEMS * 2
     return nbytes, t
+
+
+def oracle_rdfft_rate(min_seconds: float, max_tensors: int, seed0: int = 2, single_core: bool = False):
+    """GB/s of the oracle over distinct whole tensors until min_seconds of work."""
+    b_, t_, n_ = 0, 0.0, 0
+    ctx = one_core() if single_core else contextlib.nullcontext()
+    with ctx:
+        while (t_ < min_seconds or n_ == 0) and n_ < max_tensors:
+            bb, tt = oracle_tensor(seed0 + n_)
+            b_, t_, n_ = b_ + bb, t_ + tt, n_ + 1
+    return b_ / t_ / 1e9, n_, t_
+
+
+def oracle_layer_rate(B: int, D: int, p: int, seed: int, single_core: bool = False):
+    """Tokens/s of the float64 oracle's forward + backward (dense circulant matrix) at
+    (B, D, p) on bf16-valued inputs; returns (tokens/s, seconds)."""
+    import oracle
+    from synthetic import sample
+    q = D // p
+    c = sample(seed, (q, q, p), "f32", sigma=1.0 / math.sqrt(D)).exact
+    x = sample(seed + 10, (B, D), "bf16").exact
+    g = sample(seed + 20, (B, D), "bf16").exact
+    ctx = one_core() if single_core else contextlib.nullcontext()
+    with ctx:
+        t0 = time.perf_counter()
+        oracle.circ_forward(x, c)
+        oracle.circ_backward(g, x, c)
+        t = time.perf_counter() - t0
+    return B / t, t
 
 
 # --------------------------------------------------------------- reference arm
@@ -229,39 +315,237 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return 0
-    # one step: 1/8 of the 256 x 4096 tensor in each view (256 rows of p = 512 and
-    # 32 rows of p = 4096, equal bytes), forward and inverse
-    r512, r4096 = 256, 32
-    for _ in range(max(args.warmup, 0)):
-        oracle_slice(r512, r4096, seed=3)
-        break                                       # the oracle has no warm-up state
+    # the oracle keeps no state between calls, so warm-up steps only touch the code
+    for w in range(min(max(args.warmup, 0), 1)):
+        oracle_tensor(seed=2 + w)
     budget = 180.0
     total_b, total_t, steps = 0, 0.0, 0
     while steps < args.steps:
-        b, t = oracle_slice(r512, r4096, seed=3)
+        b, t = oracle_tensor(seed=2 + steps)
         total_b += b
         total_t += t
         steps += 1
         if total_t > budget:
             break
     gbs = total_b / total_t / 1e9
+    one, n1, t1 = oracle_rdfft_rate(0.0, 1, seed0=2, single_core=True)
     cores = cpu_threads()
-    sample_desc = (f"float64 oracle (O(p^2) DFT by BLAS matmul) on {steps} step(s) of 256 rows at p=512 + "
-                   f"32 rows at p=4096, forward and inverse, bf16 values; "
-                   f"{'all' if steps >= args.steps else 'stopped after'} {steps} of {args.steps} requested steps "
-                   f"(time budget {budget:.0f} s)")
+    sample_desc = (f"float64 oracle (O(p^2) DFT by BLAS matmul), forward + inverse of one whole 256x4096 "
+                   f"tensor in each view per step (2048 rows p=512 + 256 rows p=4096, bf16 values, "
+                   f"distinct seeds); {'all' if steps >= args.steps else 'stopped after'} {steps} of "
+                   f"{args.steps} requested steps (time budget {budget:.0f} s); 1 core: {one:.6f} GB/s "
+                   f"on {n1} tensor(s)")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(gbs, 6), "unit": "GB/s",
         "n_gpus": args.gpus, "steps": steps, "warmup": args.warmup, "ms_per_step": round(1e3 * total_t / steps, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "rdFFT fwd+inv of a 256x4096 N(0,1) tensor as rows of p=512 and p=4096 (bf16 values)",
-                   "slice_per_step": "256 rows p=512 + 32 rows p=4096"},
+                   "sample_per_step": "one whole tensor in each view"},
         "cpu_baseline": {"value": round(gbs, 6), "unit": "GB/s", "cores": cores, "kind": "oracle",
-                         "sample": sample_desc},
+                         "sample": sample_desc, "value_1core": round(one, 6)},
         "e2e": {"value": round(gbs, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# ------------------------------------------------------------- layer workloads
+# (name, B, D, p, seed of c): the single layer at D = 4096, p = 128 (B = 256 and 1),
+# the block-size extremes at B = 256, and one adapter of the LLaMA2-7B-shaped stack.
+LAYER_CONFIGS = (
+    ("d4096_p128_B256", 256, 4096, 128, 4),
+    ("d4096_p128_B1", 1, 4096, 128, 4),
+    ("d4096_p1024_B256", 256, 4096, 1024, 7),
+    ("d4096_p4096_B256", 256, 4096, 4096, 8),
+    ("d1024_p1024_B256", 256, 1024, 1024, 9),
+    ("d4096_p512_B4096_adapter", 4096, 4096, 512, 300),
+)
+
+
+def fft_flops(p: int) -> float:
+    """Nominal flops of one length-p real FFT (the usual 2.5 p log2 p)."""
+    return 2.5 * p * math.log2(p)
+
+
+def layer_work(B: int, D: int, p: int, s: int):
+    """Algorithmic flops and bytes of the layer's kernels at (B, D, p), s bytes per
+    activation element. The contraction of one token is q^2 packed products of p/2 - 1
+    complex bins (8 flops) and two real bins (2 flops each)."""
+    q = D // p
+    contr = q * q * (8 * (p // 2 - 1) + 4)
+    cb = 4 * q * q * p
+    x_kernel = {"flops": B * (2 * q * fft_flops(p) + contr), "bytes": 2 * B * D * s + cb}
+    gc_kernel = {"flops": B * (2 * q * fft_flops(p) + contr) + q * q * fft_flops(p), "bytes": 2 * B * D * s + cb}
+    return {
+        "fwd": x_kernel,
+        "grad_x": x_kernel,
+        "grad_c": gc_kernel,
+        # backward as the method needs it: FFT(g), FFT(x), two contractions, IFFT(grad_x),
+        # the q^2 IFFTs of grad_c; bytes g, x, c_hat, grad_x, grad_c
+        "bwd": {"flops": B * (3 * q * fft_flops(p) + 2 * contr) + q * q * fft_flops(p),
+                "bytes": 3 * B * D * s + 2 * cb},
+    }
+
+
+def run_layer_bench(rd, torch, dev, gen, hbm_peak, fp32_peak, n_sets_bytes=256 << 20):
+    """Times the layer's calls on each workload. Activations rotate over enough sets
+    that their total exceeds 2x the L2 (B = 1 excepted: a latency case), so each call
+    reads its activations from HBM; c_hat is shared, as in training."""
+    out = {}
+    dt = torch.bfloat16
+    s = 2
+    dominant = None
+    for name, B, D, p, seed in LAYER_CONFIGS:
+        q = D // p
+        per_set = 4 * B * D * s
+        nsets = 1 if B == 1 else max(2, min(64, n_sets_bytes // per_set))
+        c = torch.randn(q, q, p, device=dev, generator=gen) / D ** 0.5
+        c_hat = torch.empty_like(c)
+        gc = torch.empty_like(c)
+        sets = []
+        for _ in range(nsets):
+            sets.append({"x": torch.randn(B, D, device=dev, generator=gen).to(dt),
+                         "g": torch.randn(B, D, device=dev, generator=gen).to(dt),
+                         "y": torch.empty(B, D, device=dev, dtype=dt),
+                         "gx": torch.empty(B, D, device=dev, dtype=dt)})
+
+        calls = {
+            "prepare": lambda st: rd.circ_prepare(c, out=c_hat),
+            "fwd": lambda st: rd.circ_fwd(st["x"], c_hat, p, y=st["y"]),
+            "bwd": lambda st: rd.circ_bwd(st["g"], st["x"], c_hat, p, grad_x=st["gx"], grad_c=gc),
+            "grad_x": lambda st: rd.circ_bwd(st["g"], st["x"], c_hat, p, grad_x=st["gx"], need_grad_c=False),
+            "grad_c": lambda st: rd.circ_bwd(st["g"], st["x"], c_hat, p, grad_c=gc, need_grad_x=False),
+        }
+
+        def step_body(st):
+            rd.circ_prepare(c, out=c_hat)
+            rd.circ_fwd(st["x"], c_hat, p, y=st["y"])
+            rd.circ_bwd(st["g"], st["x"], c_hat, p, grad_x=st["gx"], grad_c=gc)
+
+        calls["fwd_bwd"] = step_body
+        times = {}
+        reps = 50 if B <= 256 else 10
+        for key, fn in calls.items():
+            g_ = graph_of(lambda fn=fn: [fn(st) for st in sets], torch)
+            times[key] = time_graph(g_, max(3, reps // nsets), torch) / nsets
+            del g_
+        work = layer_work(B, D, p, s)
+        res = {"B": B, "D": D, "p": p, "q": q,
+               "activation_sets": nsets,
+               "l2": ("activations rotate over %d sets (%.0f MiB), more than 2x L2" % (nsets, nsets * per_set / 2**20))
+                     if nsets > 1 else "one set (latency case, activations L2-resident)",
+               "fwd_tokens_s": round(B / times["fwd"], 1),
+               "bwd_tokens_s": round(B / times["bwd"], 1),
+               "fwd_bwd_tokens_s": round(B / times["fwd_bwd"], 1),
+               "fwd_bwd_us": round(1e6 * times["fwd_bwd"], 2),
+               "prepare_us": round(1e6 * times["prepare"], 2)}
+        for key in ("fwd", "bwd", "grad_x", "grad_c"):
+            t = times[key]
+            w = work[key]
+            res[key] = {"us": round(1e6 * t, 2),
+                        "GB_s": round(w["bytes"] / t / 1e9, 1),
+                        "pct_hbm": round(100 * w["bytes"] / t / 1e9 / hbm_peak, 1),
+                        "TFLOP_s": round(w["flops"] / t / 1e12, 2),
+                        "pct_fp32": round(100 * w["flops"] / t / 1e12 / fp32_peak, 1)}
+        out[name] = res
+        if name == "d4096_p128_B256":
+            # the dominant layer kernel at the D = 4096, p = 128, B = 256 workload
+            kern = max(("fwd", "grad_x", "grad_c"), key=lambda k: times[k])
+            w = work[kern]
+            dominant = {"bound": "alu", "achieved": round(w["flops"] / times[kern] / 1e12, 2),
+                        "peak": round(fp32_peak, 1), "unit": "TFLOP/s",
+                        "frac": round(w["flops"] / times[kern] / 1e12 / fp32_peak, 4), "traffic": None,
+                        "kernel": {"fwd": "k_circ_x (forward)", "grad_x": "k_circ_x (grad_x)",
+                                   "grad_c": "k_circ_gc + grad_c rdIFFT"}[kern],
+                        "workload": "D=4096 p=128 B=256 bf16",
+                        "peak_kind": "nominal FP32: SMs x 128 lanes x 2 flop x sampled SM clock",
+                        "note": "achieved = algorithmic flops of the call (FFTs 2.5 p log2 p per row, packed "
+                                "contraction 8 flops per complex bin) / its time, averaged over a CUDA graph "
+                                "of calls on rotating activations"}
+        del sets, c, c_hat, gc
+    return out, dominant
+
+
+def run_adapter_stack(rd, torch, dev, gen, world, max_over_ranks_, barrier):
+    """LLaMA2-7B-shaped stack: 32 layers x (q, v) adapters of D = 4096, p = 512, 4096
+    tokens per rank per step; every adapter's forward then every backward, grad_c of all
+    64 in one bucket all-reduced once per step (the layer's only exchange)."""
+    nl, B, D, p = 32, 4096, 4096, 512
+    q = D // p
+    dt = torch.bfloat16
+    from block_circulant_layers_b200.dp import GradCBucket
+    xs = [torch.randn(B, D, device=dev, generator=gen).to(dt) for _ in range(nl)]
+    gs = [torch.randn(B, D, device=dev, generator=gen).to(dt) for _ in range(2 * nl)]
+    cs = [torch.randn(q, q, p, device=dev, generator=gen) / D ** 0.5 for _ in range(2 * nl)]
+    chs = [torch.empty_like(c) for c in cs]
+    bucket = GradCBucket([c.shape for c in cs], device=dev)
+    gcs = bucket.views
+    ys = [torch.empty_like(xs[0]) for _ in range(2)]
+    gxs = [torch.empty_like(xs[0]) for _ in range(2)]
+
+    def stack_step():
+        for a_ in range(2 * nl):
+            rd.circ_prepare(cs[a_], out=chs[a_])
+            rd.circ_fwd(xs[a_ // 2], chs[a_], p, y=ys[a_ % 2])
+        for a_ in reversed(range(2 * nl)):
+            rd.circ_bwd(gs[a_], xs[a_ // 2], chs[a_], p, grad_x=gxs[a_ % 2], grad_c=gcs[a_])
+
+    gst = graph_of(stack_step, torch)
+    reps = 5
+    for _ in range(2):
+        gst.replay()
+        bucket.allreduce(world_size=world)
+    torch.cuda.synchronize()
+    barrier()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(reps):
+        gst.replay()
+        bucket.allreduce(world_size=world)
+    b.record()
+    torch.cuda.synchronize()
+    barrier()
+    st_t = max_over_ranks_(a.elapsed_time(b) / 1e3 / reps)
+    res = {"tokens_s": round(world * B / st_t, 1), "ms_per_step": round(1e3 * st_t, 3),
+           "tokens_per_rank": B, "adapters": 2 * nl,
+           "grad_c_allreduce_bytes": int(bucket.flat.numel() * 4) if world > 1 else 0}
+    del gst, xs, gs, cs, chs, gcs, ys, gxs, bucket
+    return res
+
+
+def layer_oracle_rates():
+    """The float64 oracle's forward + backward on the layer workloads, all cores and
+    one core: configs at B = 256 and B = 1 in full, the adapter on 64 tokens
+    (extrapolated per token)."""
+    res = {}
+    cases = (("d4096_p128_B256", 256, 4096, 128, 4, "full"),
+             ("d4096_p128_B1", 1, 4096, 128, 4, "full"),
+             ("d4096_p1024_B256", 256, 4096, 1024, 7, "full"),
+             ("d4096_p4096_B256", 256, 4096, 4096, 8, "full"),
+             ("d1024_p1024_B256", 256, 1024, 1024, 9, "full"),
+             ("d4096_p512_B4096_adapter", 64, 4096, 512, 300, "64 tokens of one adapter, extrapolated per token"))
+    for name, B, D, p, seed, how in cases:
+        r_all, t_all = oracle_layer_rate(B, D, p, seed)
+        r_one, t_one = oracle_layer_rate(B, D, p, seed, single_core=True)
+        res[name] = {"fwd_bwd_tokens_s": round(r_all, 2), "seconds": round(t_all, 3),
+                     "fwd_bwd_tokens_s_1core": round(r_one, 2), "seconds_1core": round(t_one, 3),
+                     "cores": cpu_threads(), "sample": how}
+    # the 64-adapter stack from the per-token rate of one adapter (2 adapters x 64
+    # tokens measure the same per-token cost)
+    ad = res["d4096_p512_B4096_adapter"]
+    res["llama2_7b_shape_64_adapters_tokens_s_extrapolated"] = round(ad["fwd_bwd_tokens_s"] / 64, 3)
+    # config 1: the 64 x 16 fp32 round trip
+    import oracle
+    from synthetic import sample
+    s = sample(1, (64, 16), "f32")
+    t0 = time.perf_counter()
+    n = 0
+    while time.perf_counter() - t0 < 0.2:
+        oracle.idft_packed(oracle.dft_packed(s.exact))
+        n += 1
+    res["p16_64rows_roundtrip_rows_s"] = round(64 * n / (time.perf_counter() - t0), 1)
+    return res
 
 
 # -------------------------------------------------------------------- our arm
@@ -297,56 +581,115 @@ def run_ours(args):
     gen = torch.Generator(device=dev)
     gen.manual_seed(rank_seed(rank))
     dt = torch.bfloat16
-    pools = {p: [torch.randn(ELEMS // p, p, device=dev, generator=gen).to(dt) for _ in range(POOL)] for p in PS}
+    # each view's pool is one contiguous buffer cut into POOL tensors of 256 x 4096
+    flat = {p: torch.randn(POOL * ELEMS, device=dev, generator=gen).to(dt) for p in PS}
+    pools = {p: [flat[p][i * ELEMS:(i + 1) * ELEMS].view(ELEMS // p, p) for i in range(POOL)] for p in PS}
     bytes_per_transform = 2 * ELEMS * 2             # read + write, bf16
+    fns = {"fwd": rd.rdfft_fwd, "inv": rd.rdfft_inv}
 
-    def step():
-        for p in PS:
-            fanout(lambda t, p=p: (rd.rdfft_fwd(t, p), rd.rdfft_inv(t, p)), pools[p], STREAMS, torch)
+    graphs = {}
+    with nvtx("capture"):
+        for d, p in SWEEPS:
+            graphs[(d, p)] = graph_of(
+                lambda d=d, p=p: fanout(lambda t: fns[d](t, p), pools[p], STREAMS, torch), torch)
 
-    launches_per_step = len(PS) * POOL * 2
-    bytes_per_step = launches_per_step * bytes_per_transform
-    g = graph_of(step, torch)
-    for _ in range(max(args.warmup, 3)):
-        g.replay()
-    torch.cuda.synchronize()
+    def run_round(evs=None):
+        for d, p in SWEEPS:
+            if evs is not None:
+                ev = torch.cuda.Event(enable_timing=True)
+                ev.record()
+                evs.append(((d, p), ev))
+            graphs[(d, p)].replay()
 
-    # ---- timed region: K steps, barrier + synchronize on both sides
+    with nvtx("warmup"):
+        for _ in range(max(args.warmup, 3)):
+            run_round()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(4):
+            run_round()
+        b.record()
+        torch.cuda.synchronize()
+    t_round = a.elapsed_time(b) / 1e3 / 4
+    nrep = int(max_over_ranks_(float(rounds_per_step(t_round))))
+
+    # ---- timed region: K steps of nrep rounds, barrier + synchronize on both sides
+    evs = []
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     with ClockSampler(uuid) as clk:
+        clk.wait_first()
         barrier()
         torch.cuda.synchronize()
         t_wall0 = time.time()
-        start.record()
-        for _ in range(args.steps):
-            g.replay()
-        end.record()
-        torch.cuda.synchronize()
+        with nvtx("timed"):
+            start.record()
+            for _ in range(args.steps):
+                for _ in range(nrep):
+                    run_round(evs)
+            end.record()
+            torch.cuda.synchronize()
         barrier()
         t_wall1 = time.time()
     elapsed = max_over_ranks_(start.elapsed_time(end) / 1e3)
     clocks = clk.summary(t_wall0, t_wall1)
+    launches_per_round = len(SWEEPS) * POOL
+    bytes_per_step = nrep * launches_per_round * bytes_per_transform
     value_gbs = world * bytes_per_step * args.steps / elapsed / 1e9
 
-    # ---- breakdown: each (p, direction) alone over its pool, same streams
-    def refill(p):
-        for t in pools[p]:
-            t.copy_(torch.randn(t.shape, device=dev, generator=gen).to(dt))
-
+    # per-sweep device time inside the timed region (event before each sweep)
+    sweep_t = {k: 0.0 for k in SWEEPS}
+    marks = evs + [(None, end)]
+    for (k, e0), (_, e1) in zip(marks[:-1], marks[1:]):
+        sweep_t[k] += e0.elapsed_time(e1) / 1e3
+    nsweeps = args.steps * nrep
     breakdown = {}
-    for p in PS:
-        for name, fn in (("fwd", rd.rdfft_fwd), ("inv", rd.rdfft_inv)):
-            refill(p)
-            g1 = graph_of(lambda fn=fn, p=p: fanout(lambda t: fn(t, p), pools[p], STREAMS, torch), torch)
-            t1 = time_graph(g1, 5, torch)       # few replays: a lone direction rescales the data
-            breakdown[f"bf16_p{p}_{name}"] = {
-                "GB_s": round(POOL * bytes_per_transform / t1 / 1e9, 1),
-                "us_per_launch_amortized": round(1e6 * t1 / POOL, 3),
-                "pct_hbm": round(100 * POOL * bytes_per_transform / t1 / 1e9 / hbm_peak, 1),
-            }
-            del g1
-        refill(p)
+    for d, p in SWEEPS:
+        t_launch = max_over_ranks_(sweep_t[(d, p)] / nsweeps / POOL)
+        breakdown[f"bf16_p{p}_{d}"] = {
+            "GB_s": round(bytes_per_transform / t_launch / 1e9, 1),
+            "us_per_launch_amortized": round(1e6 * t_launch, 3),
+            "pct_hbm": round(100 * bytes_per_transform / t_launch / 1e9 / hbm_peak, 1),
+            "share": round(sweep_t[(d, p)] / sum(sweep_t.values()), 4),
+        }
+    del evs, marks
+
+    # ---- roofline of the dominant kernel (largest share of the timed region)
+    dom_key = max(breakdown, key=lambda k: breakdown[k]["us_per_launch_amortized"])
+    dom = breakdown[dom_key]
+    achieved = bytes_per_transform / (dom["us_per_launch_amortized"] * 1e-6) / 1e9
+    srcs = kernel_sources_sha1()
+    traffic = None
+    if TRAFFIC_CAPTURE["sources_sha1"] == srcs:
+        traffic = TRAFFIC_CAPTURE["bytes_per_launch"].get(dom_key)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
+                "frac": round(achieved / hbm_peak, 4), "traffic": traffic, "kernel": dom_key,
+                "peak_kind": peak_kind,
+                "note": "achieved = bytes per launch (2 x 256 x 4096 x 2 B) / its amortized launch time in the "
+                        f"timed region (CUDA events around each sweep of {POOL} launches on {STREAMS} streams)"}
+
+    # ---- one large launch per kernel: the whole 256 MiB pool of a view at once
+    asym = {}
+    with nvtx("large_launch"):
+        for p in PS:
+            ts = {"fwd": [], "inv": []}
+            for _ in range(5):
+                for d in ("fwd", "inv"):
+                    a = torch.cuda.Event(enable_timing=True)
+                    b = torch.cuda.Event(enable_timing=True)
+                    a.record()
+                    fns[d](flat[p], p)
+                    b.record()
+                    torch.cuda.synchronize()
+                    ts[d].append(a.elapsed_time(b) / 1e3)
+            for d in ts:
+                t = statistics.median(ts[d])
+                asym[f"bf16_p{p}_{d}_256MiB"] = {
+                    "GB_s": round(2 * flat[p].numel() * 2 / t / 1e9, 1),
+                    "pct_hbm": round(100 * 2 * flat[p].numel() * 2 / t / 1e9 / hbm_peak, 1),
+                    "us": round(1e6 * t, 1)}
 
     # single-launch latency with a cold L2 (context for the pages' per-call ms figures);
     # forward and inverse alternate so the data keep their scale
@@ -368,20 +711,6 @@ def run_ours(args):
         for name in samples:
             lat[f"bf16_p{p}_{name}_ms"] = round(statistics.median(samples[name]), 4)
     del flush
-
-    # ---- roofline of the dominant kernel (largest share of the step)
-    dom_key = max(breakdown, key=lambda k: breakdown[k]["us_per_launch_amortized"])
-    dom = breakdown[dom_key]
-    achieved = bytes_per_transform / (dom["us_per_launch_amortized"] * 1e-6) / 1e9
-    srcs = kernel_sources_sha1()
-    traffic = None
-    if TRAFFIC_CAPTURE["sources_sha1"] == srcs:
-        traffic = TRAFFIC_CAPTURE["bytes_per_launch"].get(dom_key)
-    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm_peak, "unit": "GB/s",
-                "frac": round(achieved / hbm_peak, 4), "traffic": traffic, "kernel": dom_key,
-                "peak_kind": peak_kind,
-                "note": "achieved = bytes per launch (2 x 256 x 4096 x 2 B) / amortized launch time of "
-                        f"{POOL} launches on {STREAMS} streams"}
 
     # ---- end to end through the public API with pinned host buffers
     e2e_pool = 8
@@ -411,11 +740,12 @@ def run_ours(args):
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(e2e_reps):
-        e2e_step()
-    b.record()
-    torch.cuda.synchronize()
+    with nvtx("e2e"):
+        a.record()
+        for _ in range(e2e_reps):
+            e2e_step()
+        b.record()
+        torch.cuda.synchronize()
     barrier()
     e2e_t = max_over_ranks_(a.elapsed_time(b) / 1e3 / e2e_reps)
     e2e_bytes = len(PS) * e2e_pool * 2 * bytes_per_transform
@@ -424,139 +754,76 @@ def run_ours(args):
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": h2d,
            "note": f"{e2e_pool} tensors per view per step, each: pinned H2D copy, rdfft_fwd, rdfft_inv, D2H copy; "
                    f"tensors round-robin on {e2e_streams} streams so copies in both directions overlap the transforms"}
+    del hosts, outs
 
-    # ---- block-circulant layer tokens/s at D = 4096 (bf16)
-    layer = {}
+    # ---- block-circulant layer at D = 4096 (bf16)
+    fp32_peak = fp32_peak_tflops(clocks.get("sm_mhz"), props.multi_processor_count)
+    with nvtx("layer"):
+        layer, layer_roofline = run_layer_bench(rd, torch, dev, gen, hbm_peak, fp32_peak)
+        layer["fp32_peak_tflops"] = round(fp32_peak, 1)
+        layer["llama2_7b_shape_64_adapters_4096_tokens"] = run_adapter_stack(rd, torch, dev, gen, world,
+                                                                             max_over_ranks_, barrier)
 
-    def layer_rate(B, D, p, reps):
-        q = D // p
-        c = torch.randn(q, q, p, device=dev, generator=gen) / D ** 0.5
-        c_hat = torch.empty_like(c)
-        x = torch.randn(B, D, device=dev, generator=gen).to(dt)
-        gup = torch.randn(B, D, device=dev, generator=gen).to(dt)
-        y = torch.empty_like(x)
-        gx = torch.empty_like(x)
-        gc = torch.empty_like(c)
-
-        def body():
-            rd.circ_prepare(c, out=c_hat)
-            rd.circ_fwd(x, c_hat, p, y=y)
-            rd.circ_bwd(gup, x, c_hat, p, grad_x=gx, grad_c=gc)
-
-        gl = graph_of(body, torch)
-        tt = time_graph(gl, reps, torch)
-        return B / tt
-
-    layer["d4096_p128_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 4096, 128, 50), 1)
-    # B = 1 (one token): latency of prepare + forward + backward
-    layer["d4096_p128_B1_fwd_bwd_us"] = round(1e6 / layer_rate(1, 4096, 128, 200), 2)
-    layer["d4096_p512_B4096_fwd_bwd_tokens_s_per_adapter"] = round(layer_rate(4096, 4096, 512, 20), 1)
-    # block-size extremes, B = 256: one whole-row transform per block (q = 1) and q = 4
-    layer["d4096_p1024_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 4096, 1024, 50), 1)
-    layer["d4096_p4096_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 4096, 4096, 50), 1)
-    layer["d1024_p1024_B256_fwd_bwd_tokens_s"] = round(layer_rate(256, 1024, 1024, 50), 1)
-
-    # LLaMA2-7B-shaped adapter stack: 32 layers x (q, v) adapters, 4096 tokens per step
-    nl, B, D, p = 32, 4096, 4096, 512
-    q = D // p
-    from block_circulant_layers_b200.dp import GradCBucket
-    xs = [torch.randn(B, D, device=dev, generator=gen).to(dt) for _ in range(nl)]
-    gs = [torch.randn(B, D, device=dev, generator=gen).to(dt) for _ in range(2 * nl)]
-    cs = [torch.randn(q, q, p, device=dev, generator=gen) / D ** 0.5 for _ in range(2 * nl)]
-    chs = [torch.empty_like(c) for c in cs]
-    # the 64 grad_c live in one flat bucket: with N ranks (4096 tokens each) the step
-    # ends with one all-reduce of it, the layer's only exchange
-    bucket = GradCBucket([c.shape for c in cs], device=dev)
-    gcs = bucket.views
-    ys = [torch.empty_like(xs[0]) for _ in range(2)]
-    gxs = [torch.empty_like(xs[0]) for _ in range(2)]
-
-    def stack_step():
-        for a_ in range(2 * nl):
-            rd.circ_prepare(cs[a_], out=chs[a_])
-            rd.circ_fwd(xs[a_ // 2], chs[a_], p, y=ys[a_ % 2])
-        for a_ in reversed(range(2 * nl)):
-            rd.circ_bwd(gs[a_], xs[a_ // 2], chs[a_], p, grad_x=gxs[a_ % 2], grad_c=gcs[a_])
-
-    gst = graph_of(stack_step, torch)
-    reps = 5
-    for _ in range(2):
-        gst.replay()
-        bucket.allreduce(world_size=world)
-    torch.cuda.synchronize()
-    barrier()
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record()
-    for _ in range(reps):
-        gst.replay()
-        bucket.allreduce(world_size=world)
-    b.record()
-    torch.cuda.synchronize()
-    barrier()
-    st_t = max_over_ranks_(a.elapsed_time(b) / 1e3 / reps)
-    layer["llama2_7b_shape_64_adapters_4096_tokens_per_step_tokens_s"] = round(world * B / st_t, 1)
-    layer["llama2_7b_shape_ms_per_step"] = round(1e3 * st_t, 3)
-    layer["llama2_7b_shape_tokens_per_rank"] = B
-    layer["llama2_7b_shape_grad_c_allreduce_bytes"] = int(bucket.flat.numel() * 4) if world > 1 else 0
-    del gst
-
-    # single-layer training-step peak memory at D = 4096 through the autograd module
-    # (in-place spectrum): parameter, its gradient, activations and their gradients
-    del xs, gs, cs, chs, gcs, ys, gxs
+    # single-layer training-step peak memory at D = 4096 through the autograd module:
+    # parameter, its gradient, activations and their gradients; with the in-place
+    # spectrum (c_hat in c's own buffer) and with a temporary c_hat (the default)
     memory = {}
-    for Bm in (1, 256):
-        for pm in (128, 512, 1024, 4096):
-            torch.cuda.synchronize()
-            base = torch.cuda.memory_allocated(dev)
-            torch.cuda.reset_peak_memory_stats(dev)
-            lay = rd.BlockCirculantLinear(4096, pm, device=dev, generator=gen)
-            xm = torch.randn(Bm, 4096, device=dev, generator=gen).to(dt).requires_grad_(True)
-            ym = lay(xm)
-            ym.backward(torch.ones_like(ym))
-            torch.cuda.synchronize()
-            memory[f"B{Bm}_p{pm}_MB"] = round((torch.cuda.max_memory_allocated(dev) - base) / 1e6, 3)
-            del lay, xm, ym
+    for inplace in (True, False):
+        for Bm in (1, 256):
+            for pm in (128, 512, 1024, 4096):
+                torch.cuda.synchronize()
+                base = torch.cuda.memory_allocated(dev)
+                torch.cuda.reset_peak_memory_stats(dev)
+                lay = rd.BlockCirculantLinear(4096, pm, inplace_spectrum=inplace, device=dev, generator=gen)
+                xm = torch.randn(Bm, 4096, device=dev, generator=gen).to(dt).requires_grad_(True)
+                ym = lay(xm)
+                ym.backward(torch.ones_like(ym))
+                torch.cuda.synchronize()
+                key = f"B{Bm}_p{pm}_MB" + ("_inplace_spectrum" if inplace else "")
+                memory[key] = round((torch.cuda.max_memory_allocated(dev) - base) / 1e6, 3)
+                del lay, xm, ym
     layer["single_layer_train_step_peak_memory_d4096_bf16"] = memory
 
     # ---- 2-D rdFFT and the explicit-spectrum cast (beside the step, not in it)
     spectral = {}
-    for (n2, R2, C2, dt2, name2) in ((8, 4096, 4096, torch.bfloat16, "bf16_8x4096x4096"),
-                                     (64, 1024, 1024, torch.float32, "f32_64x1024x1024")):
-        imgs = torch.randn(n2, R2, C2, device=dev, generator=gen).to(dt2)
-        nbytes = imgs.numel() * imgs.element_size()
-        g2 = graph_of(lambda: (rd.rdfft2_fwd(imgs), rd.rdfft2_inv(imgs)), torch)
-        t2 = time_graph(g2, 10, torch)
-        gf = graph_of(lambda: rd.rdfft2_fwd(imgs), torch)
-        tf = time_graph(gf, 1, torch)                   # one forward (rescales the data once)
-        spectral[f"rdfft2_{name2}"] = {
-            "fwd_inv_ms": round(1e3 * t2, 3), "fwd_ms": round(1e3 * tf, 3),
-            "effective_GBs": round(2 * 2 * nbytes / t2 / 1e9, 1),     # read + write once per transform
-            "moved_GBs": round(2 * 4 * nbytes / t2 / 1e9, 1),         # row half + column half, each r + w
-            "note": "effective = minimum in-place traffic (read + write once) / time; the row and "
-                    "column kernels each read and write the data once"}
-        del imgs, g2, gf
-    rows_c = ELEMS // 512 * 64                      # 128 MiB packed + 128 MiB complex: above L2
-    packed = torch.randn(rows_c, 512, device=dev, generator=gen).to(dt)
-    cplx = torch.empty(rows_c, 257, 2, device=dev, dtype=dt)
-    gc2 = graph_of(lambda: rd.rdfft_to_complex(packed, 512, out=cplx), torch)
-    tc = time_graph(gc2, 20, torch)
-    spectral["to_complex_bf16_p512_GBs"] = round((packed.numel() + cplx.numel()) * 2 / tc / 1e9, 1)
-    gc3 = graph_of(lambda: rd.rdfft_from_complex(cplx, out=packed), torch)
-    tc3 = time_graph(gc3, 20, torch)
-    spectral["from_complex_bf16_p512_GBs"] = round((packed.numel() + cplx.numel()) * 2 / tc3 / 1e9, 1)
-    del packed, cplx, gc2, gc3
+    with nvtx("spectral"):
+        for (n2, R2, C2, dt2, name2) in ((8, 4096, 4096, torch.bfloat16, "bf16_8x4096x4096"),
+                                         (64, 1024, 1024, torch.float32, "f32_64x1024x1024")):
+            imgs = torch.randn(n2, R2, C2, device=dev, generator=gen).to(dt2)
+            nbytes = imgs.numel() * imgs.element_size()
+            g2 = graph_of(lambda: (rd.rdfft2_fwd(imgs), rd.rdfft2_inv(imgs)), torch)
+            t2 = time_graph(g2, 10, torch)
+            gf = graph_of(lambda: rd.rdfft2_fwd(imgs), torch)
+            tf = time_graph(gf, 1, torch)                   # one forward (rescales the data once)
+            spectral[f"rdfft2_{name2}"] = {
+                "fwd_inv_ms": round(1e3 * t2, 3), "fwd_ms": round(1e3 * tf, 3),
+                "effective_GBs": round(2 * 2 * nbytes / t2 / 1e9, 1),     # read + write once per transform
+                "moved_GBs": round(2 * 4 * nbytes / t2 / 1e9, 1),         # row half + column half, each r + w
+                "note": "effective = minimum in-place traffic (read + write once) / time; the row and "
+                        "column kernels each read and write the data once"}
+            del imgs, g2, gf
+        rows_c = ELEMS // 512 * 64                      # 128 MiB packed + 128 MiB complex: above L2
+        packed = torch.randn(rows_c, 512, device=dev, generator=gen).to(dt)
+        cplx = torch.empty(rows_c, 257, 2, device=dev, dtype=dt)
+        gc2 = graph_of(lambda: rd.rdfft_to_complex(packed, 512, out=cplx), torch)
+        tc = time_graph(gc2, 20, torch)
+        spectral["to_complex_bf16_p512_GBs"] = round((packed.numel() + cplx.numel()) * 2 / tc / 1e9, 1)
+        gc3 = graph_of(lambda: rd.rdfft_from_complex(cplx, out=packed), torch)
+        tc3 = time_graph(gc3, 20, torch)
+        spectral["from_complex_bf16_p512_GBs"] = round((packed.numel() + cplx.numel()) * 2 / tc3 / 1e9, 1)
+        del packed, cplx, gc2, gc3
 
-    # ---- CPU oracle on a bounded sample (rank 0, N = 1 only)
+    # ---- CPU oracle (rank 0, N = 1 only): the rdFFT workload and the layer workloads
     cpu = None
     if world == 1 and rank == 0:
-        b_, t_, n_ = 0, 0.0, 0
-        while t_ < 10.0 and n_ < 64:                      # about 10 s of CPU work
-            bb, tt = oracle_slice(2048, 256, seed=2 + n_)  # one whole 256 x 4096 tensor in each view
-            b_, t_, n_ = b_ + bb, t_ + tt, n_ + 1
-        cpu = {"value": round(b_ / t_ / 1e9, 6), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
-               "sample": f"float64 oracle forward + inverse of {n_} distinct 256x4096 tensors in each view "
-                         f"(2048 rows p=512, 256 rows p=4096 per tensor), {t_:.1f} s"}
+        gbs, n_, t_ = oracle_rdfft_rate(10.0, 64, seed0=2)
+        one, n1, t1 = oracle_rdfft_rate(0.0, 1, seed0=2, single_core=True)
+        cpu = {"value": round(gbs, 6), "unit": "GB/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"float64 oracle forward + inverse of {n_} distinct whole 256x4096 tensors in each view "
+                         f"(2048 rows p=512, 256 rows p=4096 per tensor), {t_:.1f} s; the reference arm times the "
+                         f"same per-tensor sample; 1 core: {one:.6f} GB/s on {n1} tensor",
+               "value_1core": round(one, 6)}
+        layer["oracle"] = layer_oracle_rates()
 
     line = {
         "metric": METRIC, "value": round(value_gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
@@ -564,21 +831,27 @@ def run_ours(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": "rdFFT fwd+inv in place, 256x4096 N(0,1) bf16 tensor as rows of p=512 and p=4096",
                    "p": list(PS), "rows": [ELEMS // p for p in PS], "pool_tensors_per_view": POOL,
-                   "streams": STREAMS, "l2": "inputs larger than L2 (256 MiB pool per rank)",
+                   "streams": STREAMS, "rounds_per_step": nrep,
+                   "step": "rounds of 4 sweeps (fwd p=512, fwd p=4096, inv p=512, inv p=4096) over the pools",
+                   "l2": "inputs larger than L2: 256 MiB pool per view; a tensor's transforms are 768 MiB "
+                         "of traffic apart",
                    "parallelism": f"dp{world} (independent rows per rank)"},
         "pct_hbm": round(100 * value_gbs / world / hbm_peak, 1),
         "roofline": roofline,
         "breakdown": breakdown,
+        "large_launch": asym,
         "single_launch_cold_ms": lat,
         "layer": layer,
+        "layer_roofline": layer_roofline,
         "spectral": spectral,
         "e2e": e2e,
         "cpu_baseline": cpu,
         "clocks": clocks,
-        "gpu_launches": launches_per_step * args.steps,
+        "gpu_launches": launches_per_round * nrep * args.steps,
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
+    del graphs
     if world > 1:
         barrier()
         dist.destroy_process_group()

@@ -8,11 +8,21 @@ given by c[i][j] (first columns, fp32). Every step of the computation runs in th
 library's kernels (rdfft_fwd / circ_fwd / circ_bwd / rdfft_inv); this file only
 marshals tensors.
 
-inplace_spectrum=True keeps no second copy of c: the spectrum c_hat is computed in
-c's own buffer (rdfft_fwd), used, and turned back into c (rdfft_inv) within the same
-forward or backward call. The round trip changes c by fp32 rounding only (relative
-error about 1e-7 per call). With inplace_spectrum=False a temporary c_hat is
-allocated by torch for each call instead.
+inplace_spectrum (default False) chooses where c_hat lives during a call:
+  * False: torch allocates a temporary fp32 c_hat (q x q x p) for each forward and
+    backward call, and c itself is never written. Exact: training sees c as the
+    optimizer left it.
+  * True: no second copy of c. The spectrum is computed in c's own buffer
+    (rdfft_fwd), used, and turned back into c (rdfft_inv) within the same call, so
+    the layer's extra memory is the activations alone (the in-place memory saving
+    the method is about). The fp32 round trip is not exact, and because it applies
+    the same rounding map to nearly the same c on every call its errors accumulate
+    linearly, not as a random walk: about 1.2e-7 relative (rms over c) per call,
+    2.5e-4 after 1000 forward + backward calls at p = 128 to 4096, measured on the
+    kernels' own arithmetic (tests/test_emulator.py) and on the GPU
+    (tests/test_layer_module_gpu.py). Use it where that drift is small against the
+    optimizer's updates. While a call runs, c holds its spectrum: work on another
+    stream must not read c until the call's stream has reached its end.
 """
 from __future__ import annotations
 
@@ -73,7 +83,7 @@ class BlockCirculantLinear(torch.nn.Module):
     or fp32; the arithmetic is fp32 and the output has the input's dtype.
     """
 
-    def __init__(self, features: int, block: int, inplace_spectrum: bool = True, device=None,
+    def __init__(self, features: int, block: int, inplace_spectrum: bool = False, device=None,
                  generator: torch.Generator | None = None):
         super().__init__()
         if block < 64 or block & (block - 1) or features % block:

@@ -191,6 +191,11 @@ int circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x, flo
  * clears that word for the current device. It synchronises with the device (a
  * cudaMemcpyFromSymbol), so call it between steps, not inside a captured graph.
  * Returns RDFFT_OK, RDFFT_ETIMEOUT, or RDFFT_ECUDA.
+ * After RDFFT_ETIMEOUT the contents of the rows of the launch that timed out are
+ * undefined, and so are those of later launches in the stream until the stream has
+ * been synchronised: a CTA whose wait gave up waits once more (again bounded) for its
+ * own copies and then exits, and a copy still in flight after that second wait may
+ * land in shared memory that a later CTA has been given.
  */
 int rdfft_take_device_error(void);
 

@@ -249,3 +249,22 @@ def test_rows_kernel_shared_memory_plan(emu, p, dtype):
         # position; the rows' staged copies start in distinct four-byte banks
         starts = [(o // 4) % 32 for o in offs]
         assert len(set(starts)) == rows, (p, dtype, starts)
+
+
+@pytest.mark.parametrize("p", [128, 512, 4096])
+def test_inplace_round_trip_drift_rate(emu, p):
+    """The layer module's in-place spectrum mode applies rdfft_fwd then rdfft_inv to the
+    fp32 parameter on every forward and backward call. Iterated, the fp32 round trip
+    drifts linearly (the same rounding map applied to nearly the same values): after
+    2000 round trips (1000 training steps without an optimizer update) the measured
+    drift is 1.2e-4 to 2.5e-4 relative rms. The bound documented for the module is
+    checked here on the kernels' own arithmetic."""
+    q = 4 if p < 1024 else 1
+    c0 = sample(5, (q * q, p), "f32", sigma=1 / 64).stored.copy()
+    c = c0.copy()
+    for _ in range(2000):
+        assert emu.rdfft_emulate(c.ctypes.data, q * q, p, 0, 0) == 0
+        assert emu.rdfft_emulate(c.ctypes.data, q * q, p, 0, 1) == 0
+    d = c.astype(np.float64) - c0
+    rms = np.sqrt(np.mean(d ** 2)) / np.sqrt(np.mean(c0.astype(np.float64) ** 2))
+    assert 1e-5 <= rms <= 5e-4, rms

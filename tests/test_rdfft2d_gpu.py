@@ -83,6 +83,25 @@ def test_2d_large_sampled_and_round_trip(rd, R, C, dtype):
         assert err <= 2 * 2e-2, err
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("C", [64, 128])
+def test_2d_r4096_every_slot(rd, C, dtype):
+    """R = 4096, where a column CTA holds W = 8 tile rows (4 left columns and their
+    mirrors): C = 64 gives 9 strips and C = 128 gives 17, the last one holding only the
+    column C/2. Every slot of the forward and of the inverse against the definition."""
+    R = 4096
+    s = sample(61_000 + C, (1, R, C), dtype)
+    t = to_device(s, dtype)
+    rd.rdfft2_fwd(t)
+    torch.cuda.synchronize()
+    assert_parity(to_host_f64(t), oracle.dft2_packed(s.exact), dtype, f"2d fwd {R}x{C}")
+    s2 = sample(62_000 + C, (1, R, C), dtype)
+    t2 = to_device(s2, dtype)
+    rd.rdfft2_inv(t2)
+    torch.cuda.synchronize()
+    assert_parity(to_host_f64(t2), oracle.idft2_packed(s2.exact), dtype, f"2d inv {R}x{C}")
+
+
 def test_2d_empty_and_neighbours_untouched(rd):
     R, C = 256, 64
     buf = torch.full((3 * R * C + 256,), 7.0, device="cuda")
