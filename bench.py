@@ -59,12 +59,13 @@ FALLBACK_HBM_GBS = 6650.0
 FP32_LANES_PER_SM = 128     # FP32 FMA lanes per B200 SM (4 sub-partitions x 32)
 NOMINAL_SM_MHZ = 1965.0
 
-ROWS_KERNEL_SOURCES = ("bulk_copy.cuh", "gen_twiddles.py", "packed_fft.cuh", "rdfft_kernels.cu", "rdfft_steps.cuh")
+ROWS_KERNEL_SOURCES = ("bulk_copy.cuh", "gen_twiddles.py", "packed_fft.cuh", "pdl.cuh", "rdfft_kernels.cu",
+                       "rdfft_steps.cuh")
 
 # ncu dram bytes per launch of the dominant kernel, with the hash of the kernel
 # sources they were captured from (see profiles/); stale counters are reported null.
-TRAFFIC_CAPTURE = {"sources_sha1": "7566fd1d3b92d0eeebfe681a79c3fb7205f22638",
-                   "bytes_per_launch": {"bf16_p4096_inv": 3444835, "bf16_p4096_fwd": 3405674}}
+TRAFFIC_CAPTURE = {"sources_sha1": "92403e3014ae4f20df38c50cae5d1a50d4b74a1d",
+                   "bytes_per_launch": {"bf16_p4096_inv": 3447984, "bf16_p4096_fwd": 3408211}}
 
 
 def kernel_sources_sha1() -> str:
@@ -447,6 +448,17 @@ def run_layer_bench(rd, torch, dev, gen, hbm_peak, fp32_peak, n_sets_bytes=256 <
                         "pct_hbm": round(100 * w["bytes"] / t / 1e9 / hbm_peak, 1),
                         "TFLOP_s": round(w["flops"] / t / 1e12, 2),
                         "pct_fp32": round(100 * w["flops"] / t / 1e12 / fp32_peak, 1)}
+        if B * D > 0 and p == 128 and D == 4096:
+            # the same forward and grad_x with the contraction on the tensor cores
+            tc = {}
+            for key, fn in (("fwd", lambda st: rd.circ_fwd_tc(st["x"], c_hat, p, y=st["y"])),
+                            ("grad_x", lambda st: rd.circ_bwd_x_tc(st["g"], c_hat, p, grad_x=st["gx"]))):
+                g_ = graph_of(lambda fn=fn: [fn(st) for st in sets], torch)
+                t = time_graph(g_, max(3, reps // nsets), torch) / nsets
+                del g_
+                tc[key] = {"us": round(1e6 * t, 2), "TFLOP_s": round(work[key]["flops"] / t / 1e12, 2),
+                           "vs_cuda_core": round(times[key] / t, 3)}
+            res["tensor_core_tcgen05"] = tc
         out[name] = res
         if name == "d4096_p128_B256":
             # the dominant layer kernel at the D = 4096, p = 128, B = 256 workload
@@ -875,7 +887,9 @@ PROFILE_CASES = {
     "circ_bwdc_d4096_p512_b4096": ("circ", (4096, 4096, 512, "bwdc")),
     "circ_fwd_d4096_p128_b256": ("circ", (256, 4096, 128, "fwd")),
     "circ_bwdc_d4096_p128_b256": ("circ", (256, 4096, 128, "bwdc")),
+    "circ_fwd_tc_d4096_p128_b256": ("circ", (256, 4096, 128, "fwd_tc")),
     "circ_step_d4096_p128_b1": ("circ_step", (1, 4096, 128)),
+    "step_round": ("step_round", ()),
 }
 
 
@@ -884,13 +898,25 @@ def run_profile_case(name: str) -> int:
 
     rows: a 160 MiB buffer (more than L2) of rows of p; rows_small: one 256 x 4096 tensor
     (the bench's per-launch size); circ: the layer kernel at (B, D, p); circ_step: the
-    layer's prepare + forward + backward at (B, D, p), every kernel of it."""
+    layer's prepare + forward + backward at (B, D, p), every kernel of it; step_round: the
+    bench's pools, one warm-up round and one round of the timed step (4 x POOL launches
+    each, issued eagerly on the same streams), for a launch list."""
     import torch
     import block_circulant_layers_b200 as rd
     kind, a = PROFILE_CASES[name]
     dev = torch.device("cuda", 0)
     gen = torch.Generator(device=dev)
     gen.manual_seed(7)
+    if kind == "step_round":
+        pools = {p: [torch.randn(ELEMS // p, p, device=dev, generator=gen).to(torch.bfloat16) for _ in range(POOL)]
+                 for p in PS}
+        fns = {"fwd": rd.rdfft_fwd, "inv": rd.rdfft_inv}
+        for _ in range(2):
+            for d, p in SWEEPS:
+                fanout(lambda t, d=d, p=p: fns[d](t, p), pools[p], STREAMS, torch)
+        torch.cuda.synchronize()
+        print(f"profile case {name}: ok")
+        return 0
     if kind == "image":
         R, C, dts, d = a
         dt = torch.bfloat16 if dts == "bf16" else torch.float32
@@ -935,6 +961,8 @@ def run_profile_case(name: str) -> int:
         for _ in range(4):
             if d == "fwd":
                 rd.circ_fwd(x, ch, p, y=y)
+            elif d == "fwd_tc":
+                rd.circ_fwd_tc(x, ch, p, y=y)
             elif d == "bwdx":
                 rd.circ_bwd(g, x, ch, p, grad_x=y, need_grad_c=False)
             else:

@@ -28,8 +28,10 @@ lib.rdfft2_fwd.argtypes = [_vp, _i64, _int, _int, _int, _vp]
 lib.rdfft2_inv.argtypes = [_vp, _i64, _int, _int, _int, _vp]
 lib.circ_fwd.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _vp]
+lib.circ_fwd_tc.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
+lib.circ_bwd_x_tc.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 for _f in (lib.rdfft_fwd, lib.rdfft_inv, lib.rdfft_to_complex, lib.rdfft_from_complex, lib.rdfft2_fwd,
-           lib.rdfft2_inv, lib.circ_fwd, lib.circ_bwd):
+           lib.rdfft2_inv, lib.circ_fwd, lib.circ_bwd, lib.circ_fwd_tc, lib.circ_bwd_x_tc):
     _f.restype = _int
 lib.rdfft_strerror.argtypes = [_int]
 lib.rdfft_strerror.restype = ctypes.c_char_p
@@ -215,6 +217,38 @@ def circ_bwd(g: torch.Tensor, x: torch.Tensor, c_hat: torch.Tensor, p: int,
         _check(lib.circ_bwd(g.data_ptr(), x.data_ptr(), c_hat.data_ptr(), gx_ptr, gc_ptr, B, D, p,
                             _dtype_code(x), _stream(x)), "circ_bwd")
     return (grad_x if need_grad_x else None), (grad_c if need_grad_c else None)
+
+
+def circ_fwd_tc(x: torch.Tensor, c_hat: torch.Tensor, p: int, y: torch.Tensor | None = None) -> torch.Tensor:
+    """circ_fwd with the per-bin contraction on the tensor cores (bf16, p = 128, D = 4096)."""
+    _cuda_dense(x, "x")
+    _cuda_dense(c_hat, "c_hat")
+    if y is None:
+        y = torch.empty_like(x)
+    _cuda_dense(y, "y")
+    if y.dtype != x.dtype or y.shape != x.shape:
+        raise ValueError("y must match x in shape and dtype")
+    B, D = _layer_dims(x, p)
+    with torch.cuda.device(x.device):
+        _check(lib.circ_fwd_tc(x.data_ptr(), c_hat.data_ptr(), y.data_ptr(), B, D, p, _dtype_code(x), _stream(x)),
+               "circ_fwd_tc")
+    return y
+
+
+def circ_bwd_x_tc(g: torch.Tensor, c_hat: torch.Tensor, p: int, grad_x: torch.Tensor | None = None) -> torch.Tensor:
+    """grad_x of circ_bwd with the per-bin contraction on the tensor cores (bf16, p = 128, D = 4096)."""
+    _cuda_dense(g, "g")
+    _cuda_dense(c_hat, "c_hat")
+    if grad_x is None:
+        grad_x = torch.empty_like(g)
+    _cuda_dense(grad_x, "grad_x")
+    if grad_x.dtype != g.dtype or grad_x.shape != g.shape:
+        raise ValueError("grad_x must match g in shape and dtype")
+    B, D = _layer_dims(g, p)
+    with torch.cuda.device(g.device):
+        _check(lib.circ_bwd_x_tc(g.data_ptr(), c_hat.data_ptr(), grad_x.data_ptr(), B, D, p, _dtype_code(g),
+                                 _stream(g)), "circ_bwd_x_tc")
+    return grad_x
 
 
 def take_device_error() -> int:

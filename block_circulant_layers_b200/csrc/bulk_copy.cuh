@@ -10,6 +10,8 @@
 
 #include <stdint.h>
 
+#include "pdl.cuh"
+
 namespace rdfft {
 
 // Error word of the kernels of the translation unit that includes this header (bit 0:
@@ -88,16 +90,5 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // finish on their own; like any write of the kernel they are visible to later work
 // in the stream once the kernel has completed.
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-
-// Programmatic dependent launch. griddep_wait() blocks until the grids this one
-// depends on (earlier work in its stream) have completed and their memory is visible;
-// a kernel launched with programmatic stream serialization calls it before its first
-// global-memory access. griddep_launch_dependents() lets the next such kernel in the
-// stream be scheduled once every CTA of this grid has called it or exited; that kernel
-// still waits in its own griddep_wait() until this grid has completed.
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() {
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
 
 }  // namespace rdfft

@@ -29,6 +29,7 @@
 #include "internal.h"
 #include "layer_policy.h"
 #include "packed_fft.cuh"
+#include "pdl.cuh"
 
 namespace rdfft {
 
@@ -145,6 +146,7 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
   const int64_t tok0 = (int64_t)blockIdx.x * TT;
   const int ntok = (int)((B - tok0) < TT ? (B - tok0) : TT);
   const int o0 = blockIdx.y * QI;            // first output block of this CTA
+  griddep_wait();                            // earlier work in the stream (c_hat, the input) is done
 
   // 1. rdFFT of the TT*q input rows (row r = t*q + b)
   fft_rows<P, NT, T>(tile, TT * q, [&](int r) -> const T* {
@@ -363,7 +365,9 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
 
   }
 
-  // 4. rdIFFT of the TT*QI output rows straight to HBM
+  // 4. rdIFFT of the TT*QI output rows straight to HBM; the next launch in the stream
+  // may be scheduled meanwhile (it waits for this grid before touching memory)
+  griddep_launch_dependents();
   ifft_rows_mirrored<P, NT, T>(tile, TT * QI, [&](int r) -> T* {
     const int t = r / QI, ol = r - t * QI;
     return t < ntok ? out + (tok0 + t) * (int64_t)D + (int64_t)(o0 + ol) * P : nullptr;
@@ -389,6 +393,7 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   // the only token slice: this CTA's sums are final and every (bin, i, j) of its group
   // is one thread-group's, so it stores them instead of adding into a zeroed grad_c
   const bool sole = (gridDim.x == 1);
+  griddep_wait();                            // earlier work in the stream (g, x, zeroed grad_c) is done
 
   if constexpr (RJ % 2 == 0) {
     // S accumulators: input blocks b and b + 1 of a group on packed fp32 pairs (RJ even),
@@ -462,6 +467,7 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
       }
     }
     // add this CTA's partial packed cross-spectrum into grad_c
+    griddep_launch_dependents();
   #pragma unroll
     for (int n = 0; n < NG; ++n) {
       const int gam = threadIdx.x + NT * n;
@@ -549,6 +555,7 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
       }
     }
     // add this CTA's partial packed cross-spectrum into grad_c
+    griddep_launch_dependents();
   #pragma unroll
     for (int n = 0; n < NG; ++n) {
       const int gam = threadIdx.x + NT * n;
@@ -604,8 +611,8 @@ static cudaError_t launch_x_cfg(const void* in, const float* chat, void* out, in
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)gx, (unsigned)(q / QI));
-  kern<<<grid, NT, smem, s>>>(static_cast<const T*>(in), chat, static_cast<T*>(out), B, q, QI);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(NT), smem, s, static_cast<const T*>(in), chat, static_cast<T*>(out), B, q,
+                    QI);
 }
 
 // Launch policy (at most 32 complex accumulators per thread, NS * TT <= 32):
@@ -660,9 +667,8 @@ static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B
     if (e != cudaSuccess) return e;
   }
   dim3 grid((unsigned)slices, (unsigned)njgroups);
-  kern<<<grid, NT, smem, s>>>(static_cast<const T*>(g), static_cast<const T*>(x), grad_c, B, q, QJ,
-                              tiles_per * TT);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, dim3(NT), smem, s, static_cast<const T*>(g), static_cast<const T*>(x), grad_c, B,
+                    q, QJ, (int64_t)(tiles_per * TT));
 }
 
 // grad_c launcher: a CTA of 512 threads keeps S for QJ input blocks in registers,

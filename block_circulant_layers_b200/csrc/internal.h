@@ -24,6 +24,13 @@ cudaError_t launch_convert(const void* in, void* out, int64_t rows, int p, int d
 // forward column transform with the pair combine, or its inverse.
 cudaError_t launch_cols(void* data, int64_t images, int R, int C, int dtype, bool inverse, cudaStream_t s);
 
+// Tensor-core (tcgen05) forward / grad_x of the layer for the shape it covers
+// (circ_tc_supported: p = 128, D = 4096, bf16; circ_fwd_tc / circ_bwd_x_tc in rdfft.h),
+// and the error word of its bounded waits.
+bool circ_tc_supported(int p, int D, int dtype);
+cudaError_t launch_circ_x_tc(const void* in, const float* chat, void* out, int64_t B, bool bwdx, cudaStream_t s);
+cudaError_t take_tc_device_error(unsigned int* flags);
+
 // Block-circulant layer forward: y = W x (see circ_fwd in rdfft.h).
 cudaError_t launch_circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p,
                             int dtype, cudaStream_t s);

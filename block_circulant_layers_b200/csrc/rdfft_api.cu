@@ -146,6 +146,32 @@ int circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x, flo
   return finish(rdfft::launch_circ_bwd(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, s));
 }
 
+int circ_fwd_tc(const void* x, const float* c_hat, void* y, int64_t B, int D, int p, int dtype,
+                rdfft_stream_t stream) {
+  if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
+  if (!layer_shape_ok(B, D, p) || !rdfft::circ_tc_supported(p, D, dtype)) return RDFFT_EINVAL;
+  if (B == 0) return RDFFT_OK;
+  if (x == nullptr || c_hat == nullptr || y == nullptr) return RDFFT_ENULL;
+  if (!aligned16(x) || !aligned16(c_hat) || !aligned16(y)) return RDFFT_EALIGN;
+  const size_t act = (size_t)B * D * 2;
+  const size_t cb = sizeof(float) * (size_t)(D / p) * (D / p) * p;
+  if (overlap(y, act, x, act) || overlap(y, act, c_hat, cb)) return RDFFT_EOVERLAP;
+  return finish(rdfft::launch_circ_x_tc(x, c_hat, y, B, false, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int circ_bwd_x_tc(const void* g, const float* c_hat, void* grad_x, int64_t B, int D, int p, int dtype,
+                  rdfft_stream_t stream) {
+  if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
+  if (!layer_shape_ok(B, D, p) || !rdfft::circ_tc_supported(p, D, dtype)) return RDFFT_EINVAL;
+  if (B == 0) return RDFFT_OK;
+  if (g == nullptr || c_hat == nullptr || grad_x == nullptr) return RDFFT_ENULL;
+  if (!aligned16(g) || !aligned16(c_hat) || !aligned16(grad_x)) return RDFFT_EALIGN;
+  const size_t act = (size_t)B * D * 2;
+  const size_t cb = sizeof(float) * (size_t)(D / p) * (D / p) * p;
+  if (overlap(grad_x, act, g, act) || overlap(grad_x, act, c_hat, cb)) return RDFFT_EOVERLAP;
+  return finish(rdfft::launch_circ_x_tc(g, c_hat, grad_x, B, true, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 const char* rdfft_strerror(int code) {
   switch (code) {
     case RDFFT_OK: return "ok";
@@ -164,10 +190,11 @@ const char* rdfft_strerror(int code) {
 }
 
 int rdfft_take_device_error(void) {
-  unsigned int flags = 0;
-  const cudaError_t e = rdfft::take_rows_device_error(&flags);
+  unsigned int flags = 0, tc_flags = 0;
+  cudaError_t e = rdfft::take_rows_device_error(&flags);
+  if (e == cudaSuccess) e = rdfft::take_tc_device_error(&tc_flags);
   if (e != cudaSuccess) return finish(e);
-  return (flags & 1u) ? RDFFT_ETIMEOUT : RDFFT_OK;
+  return ((flags | tc_flags) & 1u) ? RDFFT_ETIMEOUT : RDFFT_OK;
 }
 
 int rdfft_selftest_wait_timeout(rdfft_stream_t stream) {

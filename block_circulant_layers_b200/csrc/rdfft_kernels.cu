@@ -111,17 +111,7 @@ static cudaError_t launch_pi(T* d, int64_t rows, cudaStream_t s) {
   }
   // programmatic stream serialization: the next rows launch in the stream can be
   // scheduled while this one drains; each CTA waits (griddep_wait) before touching data
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((unsigned)grid);
-  cfg.blockDim = dim3(RowTiling<P>::THREADS);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, k_rows<P, INV, T>, d, rows);
+  return launch_pdl(k_rows<P, INV, T>, dim3((unsigned)grid), dim3(RowTiling<P>::THREADS), smem, s, d, rows);
 }
 
 template <int P, typename T>

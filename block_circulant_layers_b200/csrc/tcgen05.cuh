@@ -1,0 +1,109 @@
+// Fifth-generation tensor core (tcgen05, sm_100a) wrappers: tensor-memory allocation,
+// the single-thread MMA with shared-memory operand descriptors, its completion on an
+// mbarrier, and accumulator loads. Inline PTX, one CTA (cta_group::1), no cluster
+// multicast.
+//
+// Operand layout used here (checked on a B200 with known integer operands): tf32 A (M x K)
+// and B (N x K), both K-major, no swizzle. The matrix is cut into "core matrices" of 8
+// rows x 4 tf32 (16 bytes per row, 128 contiguous bytes); the descriptor's leading byte
+// offset (LBO) is the distance between core matrices adjacent along K, its stride byte
+// offset (SBO) the distance between 8-row groups. One MMA of kind::tf32 consumes K = 8
+// (two core matrices along K). An M = 64 accumulator puts row r at tensor-memory lane
+// 32 (r / 16) + r % 16: rows 16w..16w+15 in the first 16 lanes of the lane quarter that
+// warp w (mod 4) reads.
+#pragma once
+
+#include <stdint.h>
+
+namespace rdfft {
+namespace tc {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+// Shared-memory matrix descriptor: start address, LBO, SBO (bytes, multiples of 16),
+// descriptor version 1 (tcgen05), base offset 0, no swizzle.
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFF) >> 4);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+
+// Instruction descriptor of kind::tf32: D f32, A and B tf32, both K-major, dense.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+  return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+// Tensor-memory allocation of `ncols` columns (a power of two >= 32) by one whole warp;
+// the base address is written to *dst (shared memory).
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst)), "r"(ncols)
+               : "memory");
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D (tensor memory) = A B^T (+ D when accumulate), issued by one thread.
+__device__ __forceinline__ void mma_tf32(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives once on the mbarrier when every MMA this thread issued before has completed.
+__device__ __forceinline__ void mma_commit(uint64_t* mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(mbar))
+               : "memory");
+}
+
+// Eight consecutive 32-bit columns of this thread's tensor-memory lane (32x32b shape:
+// lane = the warp's lane quarter + lane id), waited for.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
+  uint32_t r[8];
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+               : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// Four groups of eight consecutive columns (base, base + 8, base + 16, base + 24) with
+// one wait.
+__device__ __forceinline__ void tmem_ld8x4(uint32_t taddr, float (&v)[4][8]) {
+  uint32_t r[4][8];
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r[g][0]), "=r"(r[g][1]), "=r"(r[g][2]), "=r"(r[g][3]), "=r"(r[g][4]), "=r"(r[g][5]),
+                   "=r"(r[g][6]), "=r"(r[g][7])
+                 : "r"(taddr + 8u * g));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+  for (int g = 0; g < 4; ++g)
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[g][i] = __uint_as_float(r[g][i]);
+}
+
+// Round fp32 to the tf32 grid (nearest, ties away from zero), kept in an fp32 register.
+__device__ __forceinline__ float to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+}  // namespace tc
+}  // namespace rdfft

@@ -183,11 +183,32 @@ int circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x, flo
              int64_t B, int D, int p, int dtype, rdfft_stream_t stream);
 
 /*
+ * circ_fwd_tc, circ_bwd_x_tc -- the layer's forward and grad_x (as circ_fwd, and circ_bwd
+ * with grad_c = NULL) with the per-frequency-bin contraction on the fifth-generation
+ * tensor cores: tcgen05.mma of kind::tf32 with fp32 accumulation in tensor memory.
+ * [notes] "Circulant matrix training adaptation": at bin k the sum over input blocks is
+ * a complex q x q matrix (the bin of c_hat) times each token's q-vector, i.e. a small
+ * GEMM over the tokens. Covered shape: p = 128, D = 4096 (q = 32), dtype RDFFT_BF16
+ * (tf32 operands keep 10 mantissa bits: inside the bf16 tolerance, not the fp32 one);
+ * other shapes and fp32 return RDFFT_EINVAL. Arguments, layouts and overlap rules as
+ * for circ_fwd and circ_bwd. On B200 these run slower than circ_fwd / circ_bwd at every
+ * batch size measured: the tensor cores need c_hat (q^2 p fp32, 512 KB here) staged in
+ * shared memory for every tile of four tokens, which costs more than the CUDA-core
+ * contraction it replaces. They are kept as the measured alternative.
+ */
+int circ_fwd_tc(const void* x, const float* c_hat, void* y, int64_t B, int D, int p, int dtype,
+                rdfft_stream_t stream);
+int circ_bwd_x_tc(const void* g, const float* c_hat, void* grad_x, int64_t B, int D, int p, int dtype,
+                  rdfft_stream_t stream);
+
+/*
  * rdfft_take_device_error -- the device error state of the transform kernels, then cleared.
  * No page has this; it is the library's failure detection. The row kernels move rows
  * with bulk copies and wait for them on a barrier with a bounded wait (about one
  * second): a wait that gives up leaves its rows unchanged, and records the event in a
- * word of the module's device memory instead of hanging the GPU. This call reads and
+ * word of the module's device memory instead of hanging the GPU. The tensor-core layer
+ * kernels bound their waits for the tensor cores the same way (their outputs are then
+ * left unwritten and their tensor memory is freed). This call reads and
  * clears that word for the current device. It synchronises with the device (a
  * cudaMemcpyFromSymbol), so call it between steps, not inside a captured graph.
  * Returns RDFFT_OK, RDFFT_ETIMEOUT, or RDFFT_ECUDA.

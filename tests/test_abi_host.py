@@ -31,6 +31,8 @@ def lib():
     L.rdfft2_inv.argtypes = [vp, i64, i, i, i, vp]
     L.circ_fwd.argtypes = [vp, vp, vp, i64, i, i, i, vp]
     L.circ_bwd.argtypes = [vp, vp, vp, vp, vp, i64, i, i, i, vp]
+    L.circ_fwd_tc.argtypes = [vp, vp, vp, i64, i, i, i, vp]
+    L.circ_bwd_x_tc.argtypes = [vp, vp, vp, i64, i, i, i, vp]
     L.rdfft_strerror.argtypes = [i]
     L.rdfft_strerror.restype = ctypes.c_char_p
     return L
@@ -45,7 +47,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("rdfft_fwd", "rdfft_inv", "rdfft_to_complex", "rdfft_from_complex", "rdfft2_fwd", "rdfft2_inv",
-              "circ_fwd", "circ_bwd", "rdfft_strerror", "rdfft_version", "rdfft_take_device_error",
+              "circ_fwd", "circ_bwd", "circ_fwd_tc", "circ_bwd_x_tc", "rdfft_strerror", "rdfft_version",
+              "rdfft_take_device_error",
               "rdfft_selftest_wait_timeout"):
         assert n in names
 
@@ -132,6 +135,20 @@ def test_circ_argument_errors(lib):
     assert lib.circ_bwd(A, A, Bp, A, None, 4, D, p, BF16, None) == EOVERLAP        # grad_x == g
     assert lib.circ_bwd(A, A + (1 << 25), Bp, None, A, 4, D, p, BF16, None) == EOVERLAP
     assert lib.circ_bwd(A, A + (1 << 25), Bp, A + (1 << 26), None, 4, 4000, p, BF16, None) == EINVAL
+
+
+def test_tensor_core_layer_argument_errors(lib):
+    """The tensor-core entry points check like circ_fwd and cover bf16, p = 128, D = 4096."""
+    D, p = 4096, 128
+    for f in (lib.circ_fwd_tc, lib.circ_bwd_x_tc):
+        assert f(A, Bp, A + (1 << 26), 0, D, p, BF16, None) == OK                 # empty
+        assert f(A, Bp, A + (1 << 26), 4, D, p, F32, None) == EINVAL              # fp32
+        assert f(A, Bp, A + (1 << 26), 4, 2048, p, BF16, None) == EINVAL          # D != 4096
+        assert f(A, Bp, A + (1 << 26), 4, D, 256, BF16, None) == EINVAL           # p != 128
+        assert f(A, Bp, A + (1 << 26), 4, D, p, 5, None) == EDTYPE
+        assert f(None, Bp, A, 4, D, p, BF16, None) == ENULL
+        assert f(A, Bp + 8, A + (1 << 26), 4, D, p, BF16, None) == EALIGN
+        assert f(A, Bp, A, 4, D, p, BF16, None) == EOVERLAP                       # output == input
 
 
 def test_objects_call_no_allocator():

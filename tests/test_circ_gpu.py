@@ -91,6 +91,36 @@ def test_config_d4096_p128(rd, B, dtype):
     check_all(rd, B, 4096, 128, dtype, (4, 5, 6))
 
 
+@pytest.mark.parametrize("B", [1, 2, 3, 5, 130, 256, 1027])
+def test_tensor_core_d4096_p128_bf16(rd, B):
+    """circ_fwd_tc / circ_bwd_x_tc (contraction on the tensor cores) at D = 4096, p = 128,
+    bf16, four tokens per CTA: the workload's B in {1, 256} and token counts that leave a
+    partial last CTA, every element against the oracle."""
+    D, p = 4096, 128
+    c, x, g = make_layer(B, D, p, "bf16", (4, 50 + B, 60 + B))
+    c_hat = rd.circ_prepare(to_device(c, "f32"))
+    y = rd.circ_fwd_tc(to_device(x, "bf16"), c_hat, p)
+    gx = rd.circ_bwd_x_tc(to_device(g, "bf16"), c_hat, p)
+    torch.cuda.synchronize()
+    assert_parity(to_host_f64(y), oracle.circ_forward(x.exact, c.exact), "bf16", f"tc y B={B}")
+    gx_ref, _ = oracle.circ_backward(g.exact, x.exact, c.exact)
+    assert_parity(to_host_f64(gx), gx_ref, "bf16", f"tc grad_x B={B}")
+    assert rd.take_device_error() == 0
+
+
+def test_tensor_core_shape_rules(rd):
+    """The tensor-core entry points cover bf16 at p = 128, D = 4096 only; empty is a no-op."""
+    c_hat = torch.zeros(32, 32, 128, device="cuda")
+    x = torch.zeros(2, 4096, device="cuda")
+    with pytest.raises(rd.RdfftError):
+        rd.circ_fwd_tc(x, c_hat, 128)                     # fp32
+    xb = torch.zeros(2, 2048, device="cuda", dtype=torch.bfloat16)
+    with pytest.raises(rd.RdfftError):
+        rd.circ_fwd_tc(xb, torch.zeros(16, 16, 128, device="cuda"), 128)   # D = 2048
+    e = torch.empty(0, 4096, device="cuda", dtype=torch.bfloat16)
+    assert rd.circ_fwd_tc(e, c_hat, 128).shape == (0, 4096)
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("D,p,seed", [(4096, 1024, 7), (4096, 4096, 8), (1024, 1024, 9)])
 def test_config_block_size_extremes(rd, D, p, seed, dtype):
