@@ -26,12 +26,13 @@ lib.rdfft_to_complex.argtypes = [_vp, _vp, _i64, _int, _int, _vp]
 lib.rdfft_from_complex.argtypes = [_vp, _vp, _i64, _int, _int, _vp]
 lib.rdfft2_fwd.argtypes = [_vp, _i64, _int, _int, _int, _vp]
 lib.rdfft2_inv.argtypes = [_vp, _i64, _int, _int, _int, _vp]
+lib.circ_prepare.argtypes = [_vp, _vp, _int, _int, _vp]
 lib.circ_fwd.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_fwd_tc.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_bwd_x_tc.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 for _f in (lib.rdfft_fwd, lib.rdfft_inv, lib.rdfft_to_complex, lib.rdfft_from_complex, lib.rdfft2_fwd,
-           lib.rdfft2_inv, lib.circ_fwd, lib.circ_bwd, lib.circ_fwd_tc, lib.circ_bwd_x_tc):
+           lib.rdfft2_inv, lib.circ_prepare, lib.circ_fwd, lib.circ_bwd, lib.circ_fwd_tc, lib.circ_bwd_x_tc):
     _f.restype = _int
 lib.rdfft_strerror.argtypes = [_int]
 lib.rdfft_strerror.restype = ctypes.c_char_p
@@ -159,16 +160,22 @@ def rdfft2_inv(t: torch.Tensor) -> torch.Tensor:
 
 
 def circ_prepare(c: torch.Tensor, out: torch.Tensor | None = None) -> torch.Tensor:
-    """c_hat for circ_fwd / circ_bwd: the packed rdFFT of fp32 c (q x q x p)."""
+    """c_hat for circ_fwd / circ_bwd: the packed rdFFT of fp32 c (q x q x p), computed out
+    of place into `out` (a new tensor by default; `out` may be c itself)."""
     _cuda_dense(c, "c")
     if c.dim() != 3 or c.shape[0] != c.shape[1]:
         raise ValueError("c must have shape (q, q, p)")
-    p = c.shape[2]
+    if c.dtype != torch.float32:
+        raise TypeError("c must be float32")
+    q, p = c.shape[0], c.shape[2]
     if out is None:
-        out = c.detach().to(torch.float32).clone()
-    else:
-        out.copy_(c)
-    return rdfft_fwd(out, p)
+        out = torch.empty_like(c)
+    _cuda_dense(out, "out")
+    if out.shape != c.shape or out.dtype != torch.float32:
+        raise ValueError("out must match c in shape and be float32")
+    with torch.cuda.device(c.device):
+        _check(lib.circ_prepare(c.data_ptr(), out.data_ptr(), q * p, p, _stream(c)), "circ_prepare")
+    return out
 
 
 def _layer_dims(x: torch.Tensor, p: int):

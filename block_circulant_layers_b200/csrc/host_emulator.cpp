@@ -67,7 +67,7 @@ void emu_geo(T* data, int64_t rows) {
 template <int P, bool INV, typename T>
 void emu_rows(T* data, int64_t rows, int ept) {
   if constexpr (P <= 32) {
-    for (int64_t r = 0; r < rows; ++r) row_small<P, INV, T>(data + r * P);
+    for (int64_t r = 0; r < rows; ++r) row_small<P, INV, T>(data + r * P, data + r * P);
   } else {
     if (ept == 0) {
       emu_geo<RowGeo<P>, RowTiling<P>::ROWS, INV, T>(data, rows);

@@ -10,6 +10,10 @@ namespace rdfft {
 // rows of length p; dtype 0 = fp32, 1 = bf16. Arguments are already validated.
 cudaError_t launch_rows(void* data, int64_t rows, int p, int dtype, bool inverse, cudaStream_t s);
 
+// The same transform out of place: rows read from src, written to dst (dst == src is the
+// in-place transform; any other overlap is the caller's to avoid).
+cudaError_t launch_rows_to(const void* src, void* dst, int64_t rows, int p, int dtype, bool inverse, cudaStream_t s);
+
 // Reads and clears the error word of the rows kernels (bit 0: a bounded wait timed out).
 cudaError_t take_rows_device_error(unsigned int* flags);
 

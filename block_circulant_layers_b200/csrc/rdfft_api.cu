@@ -107,6 +107,16 @@ int rdfft2_inv(void* data, int64_t images, int R, int C, int dtype, rdfft_stream
   return image_call(data, images, R, C, dtype, stream, true);
 }
 
+int circ_prepare(const float* c, float* c_hat, int D, int p, rdfft_stream_t stream) {
+  if (!layer_shape_ok(0, D, p)) return RDFFT_EINVAL;
+  if (c == nullptr || c_hat == nullptr) return RDFFT_ENULL;
+  if (!aligned16(c) || !aligned16(c_hat)) return RDFFT_EALIGN;
+  const size_t cb = sizeof(float) * (size_t)(D / p) * (D / p) * p;
+  if (c != c_hat && overlap(c, cb, c_hat, cb)) return RDFFT_EOVERLAP;
+  const int64_t rows = (int64_t)(D / p) * (D / p);
+  return finish(rdfft::launch_rows_to(c, c_hat, rows, p, RDFFT_F32, false, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 int circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p, int dtype,
              rdfft_stream_t stream) {
   if (!dtype_ok(dtype)) return RDFFT_EDTYPE;

@@ -23,18 +23,19 @@ __device__ __forceinline__ void run_steps(float* tile, int lrow, int v, RowPtr r
   }
 }
 
-// One CTA: ROWS consecutive rows. For p >= 64 the rows travel between HBM and the
-// staging buffer by bulk copies (the TMA engine, no per-element load or store
-// instructions), and the passes read their first input from and write their last
-// output to that buffer.
+// One CTA: ROWS consecutive rows, read from src and written to dst (the same rows for
+// the in-place transforms; src and dst are therefore not restrict). For p >= 64 the
+// rows travel between HBM and the staging buffer by bulk copies (the TMA engine, no
+// per-element load or store instructions), and the passes read their first input from
+// and write their last output to that buffer.
 template <int P, bool INV, typename T>
 __global__ void __launch_bounds__(RowTiling<P>::THREADS)
-k_rows(T* __restrict__ data, int64_t rows) {
+k_rows(const T* src, T* dst, int64_t rows) {
   constexpr int ROWS = RowTiling<P>::ROWS;
   griddep_wait();                                     // earlier work on these rows is done
   if constexpr (P <= 32) {
     const int64_t row = (int64_t)blockIdx.x * ROWS + threadIdx.x;
-    if (row < rows) row_small<P, INV, T>(data + row * P);
+    if (row < rows) row_small<P, INV, T>(src + row * P, dst + row * P);
     griddep_launch_dependents();
   } else {
     using G = RowGeo<P>;
@@ -50,7 +51,7 @@ k_rows(T* __restrict__ data, int64_t rows) {
       mbar_init(mbar, 1);
       mbar_arrive_expect_tx(mbar, (unsigned)(nr * SM::RAW_ROW));
       for (int r = 0; r < nr; ++r)
-        bulk_load(raw + SM::raw_off(r), data + (row0 + r) * P, SM::RAW_ROW, mbar);
+        bulk_load(raw + SM::raw_off(r), src + (row0 + r) * P, SM::RAW_ROW, mbar);
     }
     __syncthreads();                                  // the barrier exists before anyone waits
     const bool arrived = mbar_wait_bounded(mbar, 0);
@@ -67,7 +68,7 @@ k_rows(T* __restrict__ data, int64_t rows) {
     __syncthreads();
     griddep_launch_dependents();                      // the next launch may be scheduled
     if (threadIdx.x == 0) {
-      for (int r = 0; r < nr; ++r) bulk_store(data + (row0 + r) * P, raw + SM::raw_off(r), SM::RAW_ROW);
+      for (int r = 0; r < nr; ++r) bulk_store(dst + (row0 + r) * P, raw + SM::raw_off(r), SM::RAW_ROW);
       bulk_commit();
       bulk_wait_read();
     }
@@ -96,7 +97,7 @@ cudaError_t launch_wait_selftest(cudaStream_t s) {
 }
 
 template <int P, bool INV, typename T>
-static cudaError_t launch_pi(T* d, int64_t rows, cudaStream_t s) {
+static cudaError_t launch_pi(const T* src, T* d, int64_t rows, cudaStream_t s) {
   constexpr int ROWS = RowTiling<P>::ROWS;
   const int64_t grid = (rows + ROWS - 1) / ROWS;
   if (grid > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
@@ -111,37 +112,42 @@ static cudaError_t launch_pi(T* d, int64_t rows, cudaStream_t s) {
   }
   // programmatic stream serialization: the next rows launch in the stream can be
   // scheduled while this one drains; each CTA waits (griddep_wait) before touching data
-  return launch_pdl(k_rows<P, INV, T>, dim3((unsigned)grid), dim3(RowTiling<P>::THREADS), smem, s, d, rows);
+  return launch_pdl(k_rows<P, INV, T>, dim3((unsigned)grid), dim3(RowTiling<P>::THREADS), smem, s, src, d, rows);
 }
 
 template <int P, typename T>
-static cudaError_t launch_p(void* data, int64_t rows, bool inverse, cudaStream_t s) {
+static cudaError_t launch_p(const void* src, void* data, int64_t rows, bool inverse, cudaStream_t s) {
+  const T* x = static_cast<const T*>(src);
   T* d = static_cast<T*>(data);
-  return inverse ? launch_pi<P, true, T>(d, rows, s) : launch_pi<P, false, T>(d, rows, s);
+  return inverse ? launch_pi<P, true, T>(x, d, rows, s) : launch_pi<P, false, T>(x, d, rows, s);
 }
 
 template <typename T>
-static cudaError_t launch_t(void* data, int64_t rows, int p, bool inverse, cudaStream_t s) {
+static cudaError_t launch_t(const void* src, void* data, int64_t rows, int p, bool inverse, cudaStream_t s) {
   switch (p) {
-    case 2: return launch_p<2, T>(data, rows, inverse, s);
-    case 4: return launch_p<4, T>(data, rows, inverse, s);
-    case 8: return launch_p<8, T>(data, rows, inverse, s);
-    case 16: return launch_p<16, T>(data, rows, inverse, s);
-    case 32: return launch_p<32, T>(data, rows, inverse, s);
-    case 64: return launch_p<64, T>(data, rows, inverse, s);
-    case 128: return launch_p<128, T>(data, rows, inverse, s);
-    case 256: return launch_p<256, T>(data, rows, inverse, s);
-    case 512: return launch_p<512, T>(data, rows, inverse, s);
-    case 1024: return launch_p<1024, T>(data, rows, inverse, s);
-    case 2048: return launch_p<2048, T>(data, rows, inverse, s);
-    case 4096: return launch_p<4096, T>(data, rows, inverse, s);
+    case 2: return launch_p<2, T>(src, data, rows, inverse, s);
+    case 4: return launch_p<4, T>(src, data, rows, inverse, s);
+    case 8: return launch_p<8, T>(src, data, rows, inverse, s);
+    case 16: return launch_p<16, T>(src, data, rows, inverse, s);
+    case 32: return launch_p<32, T>(src, data, rows, inverse, s);
+    case 64: return launch_p<64, T>(src, data, rows, inverse, s);
+    case 128: return launch_p<128, T>(src, data, rows, inverse, s);
+    case 256: return launch_p<256, T>(src, data, rows, inverse, s);
+    case 512: return launch_p<512, T>(src, data, rows, inverse, s);
+    case 1024: return launch_p<1024, T>(src, data, rows, inverse, s);
+    case 2048: return launch_p<2048, T>(src, data, rows, inverse, s);
+    case 4096: return launch_p<4096, T>(src, data, rows, inverse, s);
     default: return cudaErrorInvalidValue;
   }
 }
 
+cudaError_t launch_rows_to(const void* src, void* dst, int64_t rows, int p, int dtype, bool inverse, cudaStream_t s) {
+  if (dtype == 0) return launch_t<float>(src, dst, rows, p, inverse, s);
+  return launch_t<bf16_t>(src, dst, rows, p, inverse, s);
+}
+
 cudaError_t launch_rows(void* data, int64_t rows, int p, int dtype, bool inverse, cudaStream_t s) {
-  if (dtype == 0) return launch_t<float>(data, rows, p, inverse, s);
-  return launch_t<bf16_t>(data, rows, p, inverse, s);
+  return launch_rows_to(data, data, rows, p, dtype, inverse, s);
 }
 
 }  // namespace rdfft

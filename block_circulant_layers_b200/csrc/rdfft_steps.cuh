@@ -40,24 +40,25 @@ RD_HD void row_step(float* tile, int lrow, int v, RowPtr rowptr, RowOk rowok) {
   }
 }
 
-// Rows of P <= 32: one thread per row, everything in registers.
+// Rows of P <= 32: one thread per row, everything in registers. The row is read from
+// src and written to dst (the same row when in place: every element is read first).
 template <int P, bool INV, typename T>
-RD_HD void row_small(T* g) {
+RD_HD void row_small(const T* src, T* dst) {
   constexpr int e = ilog2(P);
   float a[P];
   if constexpr (!INV) {
 #pragma unroll
-    for (int j = 0; j < P; ++j) a[bitrev(j, e)] = ld(g + j);
+    for (int j = 0; j < P; ++j) a[bitrev(j, e)] = ld(src + j);
     stages_contig<2, P, P, 0, false>(a);
 #pragma unroll
-    for (int j = 0; j < P; ++j) g[j] = from_f32<T>(a[j]);
+    for (int j = 0; j < P; ++j) dst[j] = from_f32<T>(a[j]);
   } else {
 #pragma unroll
-    for (int j = 0; j < P; ++j) a[j] = ld(g + j);
+    for (int j = 0; j < P; ++j) a[j] = ld(src + j);
     stages_contig<2, P, P, 0, true>(a);
     constexpr float scale = 1.0f / P;
 #pragma unroll
-    for (int j = 0; j < P; ++j) g[bitrev(j, e)] = from_f32<T>(a[j] * scale);
+    for (int j = 0; j < P; ++j) dst[bitrev(j, e)] = from_f32<T>(a[j] * scale);
   }
 }
 

@@ -139,6 +139,18 @@ int rdfft2_fwd(void* data, int64_t images, int R, int C, int dtype, rdfft_stream
 int rdfft2_inv(void* data, int64_t images, int R, int C, int dtype, rdfft_stream_t stream);
 
 /*
+ * circ_prepare -- c_hat for circ_fwd / circ_bwd: the packed rdFFT of each of the q x q
+ * circulant vectors c[i][j][:] (fp32), in one launch, out of place or in place.
+ * [notes] "Circulant matrix training adaptation": the layer multiplies by FFT(c) in the
+ * frequency domain; this computes it once per call of the layer (c changes every step).
+ *   c     : q x q x p fp32 (i = output block, j = input block), D = q p. Read only.
+ *   c_hat : q x q x p fp32, written with the packed spectra. It may be c itself (in
+ *           place); any other overlap with c returns RDFFT_EOVERLAP.
+ *   D, p  : as for circ_fwd (p a power of two in [64, 4096], D a multiple of p, <= RDFFT_MAX_D).
+ */
+int circ_prepare(const float* c, float* c_hat, int D, int p, rdfft_stream_t stream);
+
+/*
  * circ_fwd -- block-circulant linear layer, forward.
  * [notes] "Circulant matrix training adaptation": y = IFFT(FFT(c) (.) FFT(x)); the
  * product of two conjugate-symmetric spectra is conjugate symmetric, so the packed

@@ -29,6 +29,7 @@ def lib():
     L.rdfft_from_complex.argtypes = [vp, vp, i64, i, i, vp]
     L.rdfft2_fwd.argtypes = [vp, i64, i, i, i, vp]
     L.rdfft2_inv.argtypes = [vp, i64, i, i, i, vp]
+    L.circ_prepare.argtypes = [vp, vp, i, i, vp]
     L.circ_fwd.argtypes = [vp, vp, vp, i64, i, i, i, vp]
     L.circ_bwd.argtypes = [vp, vp, vp, vp, vp, i64, i, i, i, vp]
     L.circ_fwd_tc.argtypes = [vp, vp, vp, i64, i, i, i, vp]
@@ -47,7 +48,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("rdfft_fwd", "rdfft_inv", "rdfft_to_complex", "rdfft_from_complex", "rdfft2_fwd", "rdfft2_inv",
-              "circ_fwd", "circ_bwd", "circ_fwd_tc", "circ_bwd_x_tc", "rdfft_strerror", "rdfft_version",
+              "circ_prepare", "circ_fwd", "circ_bwd", "circ_fwd_tc", "circ_bwd_x_tc", "rdfft_strerror",
+              "rdfft_version",
               "rdfft_take_device_error",
               "rdfft_selftest_wait_timeout"):
         assert n in names
@@ -135,6 +137,17 @@ def test_circ_argument_errors(lib):
     assert lib.circ_bwd(A, A, Bp, A, None, 4, D, p, BF16, None) == EOVERLAP        # grad_x == g
     assert lib.circ_bwd(A, A + (1 << 25), Bp, None, A, 4, D, p, BF16, None) == EOVERLAP
     assert lib.circ_bwd(A, A + (1 << 25), Bp, A + (1 << 26), None, 4, 4000, p, BF16, None) == EINVAL
+
+
+def test_circ_prepare_argument_errors(lib):
+    D, p = 4096, 128                                   # c: 32 x 32 x 128 fp32 = 512 KiB
+    assert lib.circ_prepare(Bp, Bp + (1 << 20), D, 100, None) == EINVAL        # p not a power of two
+    assert lib.circ_prepare(Bp, Bp + (1 << 20), D, 32, None) == EINVAL         # p < 64
+    assert lib.circ_prepare(Bp, Bp + (1 << 20), 4000, p, None) == EINVAL       # D % p
+    assert lib.circ_prepare(None, Bp, D, p, None) == ENULL
+    assert lib.circ_prepare(Bp, None, D, p, None) == ENULL
+    assert lib.circ_prepare(Bp + 4, Bp + (1 << 20), D, p, None) == EALIGN
+    assert lib.circ_prepare(Bp, Bp + 4096, D, p, None) == EOVERLAP             # partial overlap
 
 
 def test_tensor_core_layer_argument_errors(lib):

@@ -91,6 +91,27 @@ def test_config_d4096_p128(rd, B, dtype):
     check_all(rd, B, 4096, 128, dtype, (4, 5, 6))
 
 
+@pytest.mark.parametrize("D,p", [(4096, 128), (1024, 1024), (4096, 4096), (256, 64)])
+def test_circ_prepare_out_of_place_and_in_place(rd, D, p):
+    """circ_prepare equals rdfft_fwd of a copy of c bit for bit, leaves c untouched, and
+    works in place (out = c); c_hat against the oracle's packed DFT."""
+    q = D // p
+    c = sample(90 + p, (q, q, p), "f32", sigma=1.0 / np.sqrt(D))
+    cd = to_device(c, "f32")
+    c0 = cd.clone()
+    ch = rd.circ_prepare(cd)
+    ref = rd.rdfft_fwd(cd.clone(), p)
+    torch.cuda.synchronize()
+    assert torch.equal(cd, c0)
+    assert torch.equal(ch, ref)
+    assert_parity(to_host_f64(ch), oracle.dft_packed(c.exact), "f32", f"c_hat p={p}")
+    same = rd.circ_prepare(cd, out=cd)
+    torch.cuda.synchronize()
+    assert same.data_ptr() == cd.data_ptr() and torch.equal(cd, ref)
+    with pytest.raises(TypeError):
+        rd.circ_prepare(c0.to(torch.bfloat16))
+
+
 @pytest.mark.parametrize("B", [1, 2, 3, 5, 130, 256, 1027])
 def test_tensor_core_d4096_p128_bf16(rd, B):
     """circ_fwd_tc / circ_bwd_x_tc (contraction on the tensor cores) at D = 4096, p = 128,
