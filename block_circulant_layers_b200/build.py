@@ -31,7 +31,7 @@ LIB = os.path.join(PKG, "librdfft.so")
 EMU = os.path.join(PKG, "librdfft_hostemu.so")
 
 CU_SOURCES = ["rdfft_api.cu", "rdfft_kernels.cu", "rdfft2d_kernels.cu", "convert_kernels.cu", "circ_launch.cu",
-              "circ_tc.cu"] + [
+              "circ_tc.cu", "circ_bwd_fused.cu"] + [
     f"circ_p{p}.cu" for p in (64, 128, 256, 512, 1024, 2048, 4096)]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -1,0 +1,272 @@
+// Block-circulant layer backward in one kernel for layers with few blocks (q <= 8):
+// grad_x and grad_c from one transform of each token's g and x.
+//
+// "Memory-Efficient Training with In-Place FFT Implementation", paper-notes page,
+// "Circulant matrix training adaptation" (gradients keep the conjugate symmetry):
+//     grad_x_j  = IFFT( sum_i conj(C_ij) (.) G_i )
+//     grad_c_ij = IFFT( sum_b G_i^b (.) conj(X_j^b) )
+// with G = rdFFT(g), X = rdFFT(x) per block, C = c_hat. circ_bwd otherwise runs two
+// kernels, each transforming g again (and grad_c also x): 32 row transforms per token
+// at q = 8. Here a persistent CTA per SM walks its slice of the tokens in tiles and,
+// per tile, transforms g and x once into its shared tile (2 q rows per token), adds
+// G conj(X) into the CTA's part of the cross-spectrum, forms the grad_x spectra over
+// the X rows, and inverse-transforms them to HBM: 24 row transforms per token.
+//
+// The cross-spectrum of the CTA (q^2 p/2 complex values, 32768 floats at p = 512,
+// q = 8: 64 per thread) lives in tensor memory, not in registers: loaded and stored
+// back (tcgen05.ld / tcgen05.st, 32x32b shape, each thread its own lane) around the
+// accumulation of each tile, it leaves the registers to the transforms and the grad_x
+// contraction. Beside it each thread keeps the c_hat values of its grad_x slots (one
+// bin, NS output blocks, all q summed blocks: 64 floats at p = 512), read from HBM once
+// per CTA instead of once per tile. At the end each CTA adds its part into grad_c (fp32 red.add into a
+// zeroed grad_c; a plain store when one CTA covers all tokens), and the caller's
+// stream runs the in-place rdIFFT of grad_c's q^2 rows after, as circ_bwd does.
+#include <cuda_runtime.h>
+
+#include "circ_kernels.cuh"
+#include "internal.h"
+#include "tcgen05.cuh"
+
+namespace rdfft {
+namespace {
+
+template <int P, int Q, typename T, int NT, int TT, int RI, int RJ>
+__global__ void __launch_bounds__(NT, 1)
+k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* __restrict__ chat,
+                 T* __restrict__ grad_x, float* __restrict__ grad_c, int64_t B, int64_t tok_per_cta) {
+  using G = LayerGeo<P>;
+  constexpr int q = Q;
+  constexpr int HB = P / 2;
+  constexpr int RJP = RJ / 2;
+  constexpr int ACC = RI * RJ * 2;                  // floats of cross-spectrum per thread
+  constexpr int NS = Q * HB / NT;                   // grad_x output blocks per thread (one bin)
+  constexpr int CH = NS * Q * 2;                    // floats of c_hat per thread
+  constexpr int PER = ACC + CH;                     // tensor-memory columns per thread
+  constexpr int WQ = NT / 128;                      // warps per tensor-memory lane quarter
+  constexpr int COLS = WQ * PER;
+  static_assert(RJ % 2 == 0 && ACC % 16 == 0 && CH % 16 == 0, "accumulator layout");
+  static_assert((COLS & (COLS - 1)) == 0 && COLS >= 32 && COLS <= 512, "tensor-memory allocation");
+  static_assert(NT % HB == 0 && NS >= 1, "the grad_x slots of a thread share one bin");
+  extern __shared__ float tile[];
+  __shared__ uint32_t tmem_holder;
+  const int D = q * P;
+  const int64_t tbeg = (int64_t)blockIdx.x * tok_per_cta;
+  const int64_t tend = (tbeg + tok_per_cta < B) ? tbeg + tok_per_cta : B;
+  const bool sole = (gridDim.x == 1);
+  const int warp = threadIdx.x >> 5;
+  const int nib = q / RI;
+  const int ng = HB * nib * (q / RJ);               // cross-spectrum groups (one per thread)
+  const int XR = TT * q;                            // first X row of the tile
+
+  griddep_wait();
+  if (warp == 0) tc::tmem_alloc(&tmem_holder, COLS);
+  tc::fence_before_sync();
+  __syncthreads();
+  tc::fence_after_sync();
+  const uint32_t tacc = tmem_holder + ((uint32_t)(32 * (warp & 3)) << 16) + (uint32_t)(PER * (warp >> 2));
+  const uint32_t tch = tacc + ACC;
+  float acc[ACC];
+#pragma unroll
+  for (int i = 0; i < ACC; ++i) acc[i] = 0.0f;
+#pragma unroll
+  for (int c = 0; c < ACC; c += 16) tc::tmem_st16(tacc + c, acc + c);
+
+  // the thread's cross-spectrum group: bin k, output blocks ib*RI.., input blocks jb*RJ..
+  const int gam = threadIdx.x;
+  const int gk = gam % HB, gib = (gam / HB) % nib, gjb = gam / HB / nib;
+  const bool gz = (gk == 0);
+  const int gkr = G::at(gk), gki = G::at(bin_im_slot<P>(gk));
+  // the thread's grad_x slots: bin xk, output blocks o_u = xo0 + u NT / HB (u < NS). Their
+  // c_hat values (for every summed block i) are the same for every token: read once here
+  // and kept in tensor memory beside the cross-spectrum, as [u][i] (re, im) pairs, with
+  // conj(c_hat) and the real pair of bin 0 folded into (a1, a2, a3, a4) at use.
+  const int xk = threadIdx.x % HB, xo0 = threadIdx.x / HB;
+  const bool xz = (xk == 0);
+  const int xkr = G::at(xk), xki = G::at(bin_im_slot<P>(xk));
+  {
+    float ch[CH];
+#pragma unroll
+    for (int u = 0; u < NS; ++u)
+#pragma unroll
+      for (int i = 0; i < Q; ++i) {
+        const float* crow = chat + (int64_t)(i * Q + xo0 + u * (NT / HB)) * P;
+        ch[2 * (u * Q + i)] = __ldg(crow + xk);
+        ch[2 * (u * Q + i) + 1] = __ldg(crow + bin_im_slot<P>(xk));
+      }
+#pragma unroll
+    for (int c = 0; c < CH; c += 16) tc::tmem_st16(tch + c, ch + c);
+  }
+  tc::tmem_wait_st();
+
+  for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
+    const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
+    if (tok0 != tbeg) __syncthreads();              // the previous tile is fully consumed
+    // 1. rdFFT of g (rows t q + i) and x (rows XR + t q + j) of the tile's tokens
+    fft_rows<P, NT, T>(tile, 2 * XR, [&](int r) -> const T* {
+      const bool isx = r >= XR;
+      const int rr = isx ? r - XR : r;
+      const int t = rr / q, b = rr - t * q;
+      if (t >= ntok) return nullptr;
+      return (isx ? x : g) + (tok0 + t) * (int64_t)D + (int64_t)b * P;
+    });
+    __syncthreads();
+
+    // 2. cross-spectrum: S_ij += G_i conj(X_j) over the tile's tokens, from and back to
+    // tensor memory; input blocks b and b + 1 on packed fp32 pairs
+#pragma unroll
+    for (int c = 0; c < ACC; c += 16) tc::tmem_ld16_nowait(tacc + c, acc + c);
+    tc::tmem_wait_ld();
+    if (gam < ng) {
+      for (int t = 0; t < ntok; ++t) {
+        float gr[RI], gi[RI];
+#pragma unroll
+        for (int a = 0; a < RI; ++a) {
+          const int rb = G::row_base(t * q + gib * RI + a);
+          gr[a] = tile[rb + gkr];
+          gi[a] = tile[rb + gki];
+        }
+#pragma unroll
+        for (int bp = 0; bp < RJP; ++bp) {
+          float xr[2], xi[2];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int rb = G::row_base(XR + t * q + gjb * RJ + 2 * bp + h);
+            xr[h] = tile[rb + gkr];
+            xi[h] = tile[rb + gki];
+          }
+          // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)
+          const f2 vxr = f2_mk(xr[0], xr[1]);
+          const f2 vxi_re = gz ? f2_bc(0.0f) : f2_mk(xi[0], xi[1]);
+          const f2 vx_im = gz ? f2_mk(xi[0], xi[1]) : f2_mk(xr[0], xr[1]);
+          const f2 vxi_im = gz ? f2_bc(0.0f) : f2_mk(-xi[0], -xi[1]);
+#pragma unroll
+          for (int a = 0; a < RI; ++a) {
+            const int o = (a * RJP + bp) * 4;
+            const f2 vgr = f2_bc(gr[a]), vgi = f2_bc(gi[a]);
+            const f2 sr = f2_fma(vgr, vxr, f2_fma(vgi, vxi_re, f2_mk(acc[o], acc[o + 1])));
+            const f2 si = f2_fma(vgi, vx_im, f2_fma(vgr, vxi_im, f2_mk(acc[o + 2], acc[o + 3])));
+            acc[o] = sr.x;
+            acc[o + 1] = sr.y;
+            acc[o + 2] = si.x;
+            acc[o + 3] = si.y;
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < ACC; c += 16) tc::tmem_st16(tacc + c, acc + c);
+    tc::tmem_wait_st();
+    __syncthreads();                                 // X rows read: they become grad_x rows
+
+    // 3. grad_x spectra over the X rows: Y_j = sum_i conj(C_ij) G_i, stored mirrored
+    // (slot k = Re - Im, slot p - k = Re + Im; bin 0 keeps its real pair)
+    {
+      float ch[CH];
+#pragma unroll
+      for (int c = 0; c < CH; c += 16) tc::tmem_ld16_nowait(tch + c, ch + c);
+      tc::tmem_wait_ld();
+#pragma unroll
+      for (int u = 0; u < NS; ++u) {
+        const int o = xo0 + u * (NT / HB);
+        float yr[TT], yi[TT];
+#pragma unroll
+        for (int t = 0; t < TT; ++t) yr[t] = yi[t] = 0.0f;
+#pragma unroll
+        for (int i = 0; i < Q; ++i) {
+          const float cr = ch[2 * (u * Q + i)], ci = ch[2 * (u * Q + i) + 1];
+          const float a2 = xz ? 0.0f : ci, a3 = xz ? ci : cr, a4 = xz ? 0.0f : -ci;
+#pragma unroll
+          for (int t = 0; t < TT; ++t) {
+            if (t < ntok) {
+              const int rb = G::row_base(t * Q + i);
+              const float gr = tile[rb + xkr], gi = tile[rb + xki];
+              yr[t] = fmaf(cr, gr, fmaf(a2, gi, yr[t]));
+              yi[t] = fmaf(a3, gi, fmaf(a4, gr, yi[t]));
+            }
+          }
+        }
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          if (t < ntok) {
+            const int rb = G::row_base(XR + t * Q + o);
+            tile[rb + xkr] = xz ? yr[t] : yr[t] - yi[t];
+            tile[rb + xki] = xz ? yi[t] : yr[t] + yi[t];
+          }
+        }
+      }
+    }
+    __syncthreads();
+    // 4. rdIFFT (Hartley form) of the grad_x rows straight to HBM
+    ifft_rows_mirrored<P, NT, T>(tile + G::row_base(XR), XR, [&](int r) -> T* {
+      const int t = r / q, j = r - t * q;
+      return t < ntok ? grad_x + (tok0 + t) * (int64_t)D + (int64_t)j * P : nullptr;
+    });
+  }
+
+  // 5. the CTA's cross-spectrum into grad_c
+  griddep_launch_dependents();
+#pragma unroll
+  for (int c = 0; c < ACC; c += 16) tc::tmem_ld16_nowait(tacc + c, acc + c);
+  tc::tmem_wait_ld();
+  if (gam < ng) {
+    const int kim = bin_im_slot<P>(gk);
+#pragma unroll
+    for (int a = 0; a < RI; ++a)
+#pragma unroll
+      for (int b = 0; b < RJ; ++b) {
+        float* dst = grad_c + ((int64_t)(gib * RI + a) * q + (gjb * RJ + b)) * P;
+        const int o = (a * RJP + b / 2) * 4 + (b & 1);
+        const float vr = acc[o], vi = acc[o + 2];
+        if (sole) {
+          dst[gk] = vr;
+          dst[kim] = vi;
+        } else {
+          atomicAdd(dst + gk, vr);
+          atomicAdd(dst + kim, vi);
+        }
+      }
+  }
+  tc::fence_before_sync();
+  __syncthreads();
+  if (warp == 0) tc::tmem_dealloc(tmem_holder, COLS);
+}
+
+template <int P, int Q, typename T, int TT, int RI, int RJ>
+cudaError_t run_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B,
+                      cudaStream_t s) {
+  constexpr int NT = 512;
+  constexpr int q = Q;
+  auto kern = k_circ_bwd_fused<P, Q, T, NT, TT, RI, RJ>;
+  const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(2 * TT * q);
+  cudaError_t e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  int64_t tiles_per = 1;
+  const int slices = layer_gc_slices(1, (B + TT - 1) / TT, num_sms(), &tiles_per);
+  if (slices > 1) {
+    e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)q * q * P, s);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(kern, dim3((unsigned)slices), dim3(NT), smem, s, static_cast<const T*>(g),
+                    static_cast<const T*>(x), chat, static_cast<T*>(grad_x), grad_c, B, (int64_t)(tiles_per * TT));
+}
+
+template <typename T>
+cudaError_t fused_t(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B, int q,
+                    int p, cudaStream_t s) {
+  if (p == 512 && q == 8) return run_fused<512, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s);
+  if (p == 1024 && q == 4) return run_fused<1024, 4, T, 2, 4, 4>(g, x, chat, grad_x, grad_c, B, s);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+bool circ_bwd_fused_supported(int p, int D) { return (p == 512 && D == 4096) || (p == 1024 && D == 4096); }
+
+cudaError_t launch_circ_bwd_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c,
+                                  int64_t B, int D, int p, int dtype, cudaStream_t s) {
+  const int q = D / p;
+  if (dtype == 0) return fused_t<float>(g, x, chat, grad_x, grad_c, B, q, p, s);
+  return fused_t<bf16_t>(g, x, chat, grad_x, grad_c, B, q, p, s);
+}
+
+}  // namespace rdfft

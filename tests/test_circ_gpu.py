@@ -91,6 +91,32 @@ def test_config_d4096_p128(rd, B, dtype):
     check_all(rd, B, 4096, 128, dtype, (4, 5, 6))
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B", [1, 3, 5, 9, 37])
+@pytest.mark.parametrize("p", [512, 1024])
+def test_fused_backward_shapes(rd, p, B, dtype):
+    """D = 4096 at p = 512 (q = 8) and p = 1024 (q = 4): circ_bwd computes grad_x and grad_c
+    in one kernel (the cross-spectrum accumulated in tensor memory). Ragged token counts:
+    one CTA storing grad_c, and several adding into it."""
+    check_all(rd, B, 4096, p, dtype, (110 + p, 120 + B, 130 + B))
+
+
+@pytest.mark.parametrize("p", [512, 1024])
+def test_fused_backward_stores_every_grad_c_element(rd, p):
+    """With a single CTA (few tokens) the fused kernel stores grad_c instead of adding into a
+    zeroed buffer: a grad_c full of NaN must come out finite and right."""
+    B, D = 3, 4096
+    c, x, g = make_layer(B, D, p, "bf16", (140, 141, 142))
+    c_hat = rd.circ_prepare(to_device(c, "f32"))
+    gc = torch.full(c_hat.shape, float("nan"), device="cuda")
+    gx = torch.empty(B, D, device="cuda", dtype=torch.bfloat16)
+    rd.circ_bwd(to_device(g, "bf16"), to_device(x, "bf16"), c_hat, p, grad_x=gx, grad_c=gc)
+    torch.cuda.synchronize()
+    gx_ref, gc_ref = oracle.circ_backward(g.exact, x.exact, c.exact)
+    assert_parity(to_host_f64(gc), gc_ref, "bf16", "fused grad_c from NaN")
+    assert_parity(to_host_f64(gx), gx_ref, "bf16", "fused grad_x")
+
+
 @pytest.mark.parametrize("D,p", [(4096, 128), (1024, 1024), (4096, 4096), (256, 64)])
 def test_circ_prepare_out_of_place_and_in_place(rd, D, p):
     """circ_prepare equals rdfft_fwd of a copy of c bit for bit, leaves c untouched, and
