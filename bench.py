@@ -888,6 +888,7 @@ PROFILE_CASES = {
     "circ_fwd_d4096_p128_b256": ("circ", (256, 4096, 128, "fwd")),
     "circ_bwdc_d4096_p128_b256": ("circ", (256, 4096, 128, "bwdc")),
     "circ_fwd_tc_d4096_p128_b256": ("circ", (256, 4096, 128, "fwd_tc")),
+    "circ_bwd_d4096_p512_b4096": ("circ", (4096, 4096, 512, "bwd")),
     "circ_step_d4096_p128_b1": ("circ_step", (1, 4096, 128)),
     "step_round": ("step_round", ()),
 }
@@ -963,6 +964,8 @@ def run_profile_case(name: str) -> int:
                 rd.circ_fwd(x, ch, p, y=y)
             elif d == "fwd_tc":
                 rd.circ_fwd_tc(x, ch, p, y=y)
+            elif d == "bwd":
+                rd.circ_bwd(g, x, ch, p, grad_x=y, grad_c=gc)
             elif d == "bwdx":
                 rd.circ_bwd(g, x, ch, p, grad_x=y, need_grad_c=False)
             else:

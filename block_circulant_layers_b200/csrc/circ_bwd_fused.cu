@@ -78,8 +78,8 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
   const int gkr = G::at(gk), gki = G::at(bin_im_slot<P>(gk));
   // the thread's grad_x slots: bin xk, output blocks o_u = xo0 + u NT / HB (u < NS). Their
   // c_hat values (for every summed block i) are the same for every token: read once here
-  // and kept in tensor memory beside the cross-spectrum, as [u][i] (re, im) pairs, with
-  // conj(c_hat) and the real pair of bin 0 folded into (a1, a2, a3, a4) at use.
+  // and kept in tensor memory beside the cross-spectrum, as [i][u] (re, im) pairs (16
+  // columns = two summed blocks), with conj(c_hat) and bin 0's real pair applied at use.
   const int xk = threadIdx.x % HB, xo0 = threadIdx.x / HB;
   const bool xz = (xk == 0);
   const int xkr = G::at(xk), xki = G::at(bin_im_slot<P>(xk));
@@ -90,8 +90,8 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
 #pragma unroll
       for (int i = 0; i < Q; ++i) {
         const float* crow = chat + (int64_t)(i * Q + xo0 + u * (NT / HB)) * P;
-        ch[2 * (u * Q + i)] = __ldg(crow + xk);
-        ch[2 * (u * Q + i) + 1] = __ldg(crow + bin_im_slot<P>(xk));
+        ch[2 * (i * NS + u)] = __ldg(crow + xk);
+        ch[2 * (i * NS + u) + 1] = __ldg(crow + bin_im_slot<P>(xk));
       }
 #pragma unroll
     for (int c = 0; c < CH; c += 16) tc::tmem_st16(tch + c, ch + c);
@@ -161,36 +161,57 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
     // 3. grad_x spectra over the X rows: Y_j = sum_i conj(C_ij) G_i, stored mirrored
     // (slot k = Re - Im, slot p - k = Re + Im; bin 0 keeps its real pair)
     {
-      float ch[CH];
+      // all NS slots share the bin, so each G value is read once for all of them; slot
+      // pairs (u, u + 1) accumulate on packed fp32 pairs
+      static_assert(NS % 2 == 0 && 2 * NS == 8 && Q % 2 == 0, "slot pairs; two summed blocks per 16 columns");
+      f2 yr[NS / 2][TT], yi[NS / 2][TT];
 #pragma unroll
-      for (int c = 0; c < CH; c += 16) tc::tmem_ld16_nowait(tch + c, ch + c);
-      tc::tmem_wait_ld();
+      for (int w = 0; w < NS / 2; ++w)
 #pragma unroll
-      for (int u = 0; u < NS; ++u) {
-        const int o = xo0 + u * (NT / HB);
-        float yr[TT], yi[TT];
+        for (int t = 0; t < TT; ++t) yr[w][t] = yi[w][t] = f2_bc(0.0f);
+      float ch[16];
 #pragma unroll
-        for (int t = 0; t < TT; ++t) yr[t] = yi[t] = 0.0f;
+      for (int i = 0; i < Q; ++i) {
+        if ((i & 1) == 0) {
+          tc::tmem_ld16_nowait(tch + 2 * i * NS, ch);
+          tc::tmem_wait_ld();
+        }
+        const int cb = 2 * (i & 1) * NS;
+        f2 c1[NS / 2], c2[NS / 2], c3[NS / 2], c4[NS / 2];
 #pragma unroll
-        for (int i = 0; i < Q; ++i) {
-          const float cr = ch[2 * (u * Q + i)], ci = ch[2 * (u * Q + i) + 1];
-          const float a2 = xz ? 0.0f : ci, a3 = xz ? ci : cr, a4 = xz ? 0.0f : -ci;
-#pragma unroll
-          for (int t = 0; t < TT; ++t) {
-            if (t < ntok) {
-              const int rb = G::row_base(t * Q + i);
-              const float gr = tile[rb + xkr], gi = tile[rb + xki];
-              yr[t] = fmaf(cr, gr, fmaf(a2, gi, yr[t]));
-              yi[t] = fmaf(a3, gi, fmaf(a4, gr, yi[t]));
-            }
-          }
+        for (int w = 0; w < NS / 2; ++w) {
+          const float cr0 = ch[cb + 4 * w], ci0 = ch[cb + 4 * w + 1];
+          const float cr1 = ch[cb + 4 * w + 2], ci1 = ch[cb + 4 * w + 3];
+          // conj(c) G: re = cr gr + ci gi, im = cr gi - ci gr; bin 0: (cr gr, ci gi)
+          c1[w] = f2_mk(cr0, cr1);
+          c2[w] = xz ? f2_bc(0.0f) : f2_mk(ci0, ci1);
+          c3[w] = xz ? f2_mk(ci0, ci1) : f2_mk(cr0, cr1);
+          c4[w] = xz ? f2_bc(0.0f) : f2_mk(-ci0, -ci1);
         }
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
           if (t < ntok) {
+            const int rb = G::row_base(t * Q + i);
+            const f2 gr = f2_bc(tile[rb + xkr]), gi = f2_bc(tile[rb + xki]);
+#pragma unroll
+            for (int w = 0; w < NS / 2; ++w) {
+              yr[w][t] = f2_fma(c1[w], gr, f2_fma(c2[w], gi, yr[w][t]));
+              yi[w][t] = f2_fma(c3[w], gi, f2_fma(c4[w], gr, yi[w][t]));
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < NS; ++u) {
+        const int o = xo0 + u * (NT / HB);
+#pragma unroll
+        for (int t = 0; t < TT; ++t) {
+          if (t < ntok) {
+            const float ar = (u & 1) ? yr[u / 2][t].y : yr[u / 2][t].x;
+            const float ai = (u & 1) ? yi[u / 2][t].y : yi[u / 2][t].x;
             const int rb = G::row_base(XR + t * Q + o);
-            tile[rb + xkr] = xz ? yr[t] : yr[t] - yi[t];
-            tile[rb + xki] = xz ? yi[t] : yr[t] + yi[t];
+            tile[rb + xkr] = xz ? ar : ar - ai;
+            tile[rb + xki] = xz ? ai : ar + ai;
           }
         }
       }
