@@ -74,14 +74,17 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
   // the thread's cross-spectrum group: bin k, output blocks ib*RI.., input blocks jb*RJ..
   const int gam = threadIdx.x;
   const int gk = gam % HB, gib = (gam / HB) % nib, gjb = gam / HB / nib;
-  const bool gz = (gk == 0);
+  // a warp holds bin 0 (grad_c group or grad_x slot) only if its first lane does; such
+  // warps take the real pair's component-wise products, the others the complex ones
+  const bool warp_bin0 = (threadIdx.x & ~31u) % HB == 0;
   const int gkr = G::at(gk), gki = G::at(bin_im_slot<P>(gk));
   // the thread's grad_x slots: bin xk, output blocks o_u = xo0 + u NT / HB (u < NS). Their
   // c_hat values (for every summed block i) are the same for every token: read once here
-  // and kept in tensor memory beside the cross-spectrum, as [i][u] (re, im) pairs (16
-  // columns = two summed blocks), with conj(c_hat) and bin 0's real pair applied at use.
+  // and kept in tensor memory beside the cross-spectrum, as [i][slot pair w] (re_2w,
+  // re_2w+1, im_2w, im_2w+1) (16 columns = two summed blocks), with conj(c_hat) and bin 0's
+  // real pair applied at use.
+  constexpr int XG = NT / HB;
   const int xk = threadIdx.x % HB, xo0 = threadIdx.x / HB;
-  const bool xz = (xk == 0);
   const int xkr = G::at(xk), xki = G::at(bin_im_slot<P>(xk));
   {
     float ch[CH];
@@ -89,9 +92,10 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
     for (int u = 0; u < NS; ++u)
 #pragma unroll
       for (int i = 0; i < Q; ++i) {
-        const float* crow = chat + (int64_t)(i * Q + xo0 + u * (NT / HB)) * P;
-        ch[2 * (i * NS + u)] = __ldg(crow + xk);
-        ch[2 * (i * NS + u) + 1] = __ldg(crow + bin_im_slot<P>(xk));
+        const float* crow = chat + (int64_t)(i * Q + xo0 + u * XG) * P;
+        const int c = 2 * (i * NS + (u & ~1)) + (u & 1);
+        ch[c] = __ldg(crow + xk);
+        ch[c + 2] = __ldg(crow + bin_im_slot<P>(xk));
       }
 #pragma unroll
     for (int c = 0; c < CH; c += 16) tc::tmem_st16(tch + c, ch + c);
@@ -116,7 +120,11 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
 #pragma unroll
     for (int c = 0; c < ACC; c += 16) tc::tmem_ld16_nowait(tacc + c, acc + c);
     tc::tmem_wait_ld();
-    if (gam < ng) {
+    // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0 (real pair): (gr xr, gi xi),
+    // written as re += gr xr + gi xa, im += gi xb + gr xc with the x terms chosen per
+    // input-block pair; bin0 = false (warps with no bin-0 group) drops the selects
+    auto accumulate = [&](bool bin0) {
+      const bool gz = bin0 && (gk == 0);
       for (int t = 0; t < ntok; ++t) {
         float gr[RI], gi[RI];
 #pragma unroll
@@ -134,17 +142,16 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
             xr[h] = tile[rb + gkr];
             xi[h] = tile[rb + gki];
           }
-          // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)
           const f2 vxr = f2_mk(xr[0], xr[1]);
-          const f2 vxi_re = gz ? f2_bc(0.0f) : f2_mk(xi[0], xi[1]);
-          const f2 vx_im = gz ? f2_mk(xi[0], xi[1]) : f2_mk(xr[0], xr[1]);
-          const f2 vxi_im = gz ? f2_bc(0.0f) : f2_mk(-xi[0], -xi[1]);
+          const f2 vxa = gz ? f2_bc(0.0f) : f2_mk(xi[0], xi[1]);
+          const f2 vxb = gz ? f2_mk(xi[0], xi[1]) : vxr;
+          const f2 vxc = gz ? f2_bc(0.0f) : f2_mk(-xi[0], -xi[1]);
 #pragma unroll
           for (int a = 0; a < RI; ++a) {
             const int o = (a * RJP + bp) * 4;
             const f2 vgr = f2_bc(gr[a]), vgi = f2_bc(gi[a]);
-            const f2 sr = f2_fma(vgr, vxr, f2_fma(vgi, vxi_re, f2_mk(acc[o], acc[o + 1])));
-            const f2 si = f2_fma(vgi, vx_im, f2_fma(vgr, vxi_im, f2_mk(acc[o + 2], acc[o + 3])));
+            const f2 sr = f2_fma(vgr, vxr, f2_fma(vgi, vxa, f2_mk(acc[o], acc[o + 1])));
+            const f2 si = f2_fma(vgi, vxb, f2_fma(vgr, vxc, f2_mk(acc[o + 2], acc[o + 3])));
             acc[o] = sr.x;
             acc[o + 1] = sr.y;
             acc[o + 2] = si.x;
@@ -152,6 +159,10 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
           }
         }
       }
+    };
+    if (gam < ng) {
+      if (warp_bin0) accumulate(true);               // warp-uniform: each side is specialised
+      else accumulate(false);
     }
 #pragma unroll
     for (int c = 0; c < ACC; c += 16) tc::tmem_st16(tacc + c, acc + c);
@@ -169,49 +180,55 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
       for (int w = 0; w < NS / 2; ++w)
 #pragma unroll
         for (int t = 0; t < TT; ++t) yr[w][t] = yi[w][t] = f2_bc(0.0f);
-      float ch[16];
+      // conj(c) G as yr += cr xa + ci xb, yi += cr xc + ci xd with the token's G terms
+      //   complex bin: xa = gr, xb = gi, xc = gi, xd = -gr;  bin 0: xa = gr, xb = xc = 0, xd = gi
+      auto contract = [&](bool bin0) {
+        const bool xz = bin0 && (xk == 0);
+        float ch[16];
 #pragma unroll
-      for (int i = 0; i < Q; ++i) {
-        if ((i & 1) == 0) {
-          tc::tmem_ld16_nowait(tch + 2 * i * NS, ch);
-          tc::tmem_wait_ld();
-        }
-        const int cb = 2 * (i & 1) * NS;
-        f2 c1[NS / 2], c2[NS / 2], c3[NS / 2], c4[NS / 2];
+        for (int i = 0; i < Q; ++i) {
+          if ((i & 1) == 0) {
+            tc::tmem_ld16_nowait(tch + 2 * i * NS, ch);
+            tc::tmem_wait_ld();
+          }
+          const int cb = 2 * (i & 1) * NS;
+          f2 cr[NS / 2], ci[NS / 2];
 #pragma unroll
-        for (int w = 0; w < NS / 2; ++w) {
-          const float cr0 = ch[cb + 4 * w], ci0 = ch[cb + 4 * w + 1];
-          const float cr1 = ch[cb + 4 * w + 2], ci1 = ch[cb + 4 * w + 3];
-          // conj(c) G: re = cr gr + ci gi, im = cr gi - ci gr; bin 0: (cr gr, ci gi)
-          c1[w] = f2_mk(cr0, cr1);
-          c2[w] = xz ? f2_bc(0.0f) : f2_mk(ci0, ci1);
-          c3[w] = xz ? f2_mk(ci0, ci1) : f2_mk(cr0, cr1);
-          c4[w] = xz ? f2_bc(0.0f) : f2_mk(-ci0, -ci1);
-        }
+          for (int w = 0; w < NS / 2; ++w) {
+            cr[w] = f2_mk(ch[cb + 4 * w], ch[cb + 4 * w + 1]);
+            ci[w] = f2_mk(ch[cb + 4 * w + 2], ch[cb + 4 * w + 3]);
+          }
 #pragma unroll
-        for (int t = 0; t < TT; ++t) {
-          if (t < ntok) {
-            const int rb = G::row_base(t * Q + i);
-            const f2 gr = f2_bc(tile[rb + xkr]), gi = f2_bc(tile[rb + xki]);
+          for (int t = 0; t < TT; ++t) {
+            if (t < ntok) {
+              const int rb = G::row_base(t * Q + i);
+              const float vr = tile[rb + xkr], vi = tile[rb + xki];
+              const f2 xa = f2_bc(vr);
+              const f2 xb = f2_bc(xz ? 0.0f : vi);
+              const f2 xc = xb;
+              const f2 xd = f2_bc(xz ? vi : -vr);
 #pragma unroll
-            for (int w = 0; w < NS / 2; ++w) {
-              yr[w][t] = f2_fma(c1[w], gr, f2_fma(c2[w], gi, yr[w][t]));
-              yi[w][t] = f2_fma(c3[w], gi, f2_fma(c4[w], gr, yi[w][t]));
+              for (int w = 0; w < NS / 2; ++w) {
+                yr[w][t] = f2_fma(cr[w], xa, f2_fma(ci[w], xb, yr[w][t]));
+                yi[w][t] = f2_fma(cr[w], xc, f2_fma(ci[w], xd, yi[w][t]));
+              }
             }
           }
         }
-      }
+      };
+      if (warp_bin0) contract(true);                 // warp-uniform: each side is specialised
+      else contract(false);
 #pragma unroll
       for (int u = 0; u < NS; ++u) {
-        const int o = xo0 + u * (NT / HB);
+        const int o = xo0 + u * XG;
 #pragma unroll
         for (int t = 0; t < TT; ++t) {
           if (t < ntok) {
             const float ar = (u & 1) ? yr[u / 2][t].y : yr[u / 2][t].x;
             const float ai = (u & 1) ? yi[u / 2][t].y : yi[u / 2][t].x;
             const int rb = G::row_base(XR + t * Q + o);
-            tile[rb + xkr] = xz ? ar : ar - ai;
-            tile[rb + xki] = xz ? ai : ar + ai;
+            tile[rb + xkr] = xk == 0 ? ar : ar - ai;
+            tile[rb + xki] = xk == 0 ? ai : ar + ai;
           }
         }
       }

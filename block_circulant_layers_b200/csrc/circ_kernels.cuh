@@ -159,25 +159,25 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
   // (NT a multiple of p/2, i.e. p <= 512), slot pairs run on packed fp32 pairs; with a
   // bin per slot (p >= 1024) pairing saves no loads and costs registers, so it is scalar.
   if constexpr (NT % (P / 2) == 0 && NS >= 2) {
-    // 2. contraction: thread slot s covers bin k and output block ol of all TT tokens.
-    // Slots are taken in pairs (s, s + 1) on packed fp32 pairs: each pair accumulates
-    // two output blocks (two bins at p >= 1024) of one token in one FFMA2 per term.
+    // 2. contraction: thread slot s covers bin k = tid % (p/2) and output block
+    // ol = w + G s (w = tid / (p/2), G = NT / (p/2) slot groups) of all TT tokens. Slots
+    // are taken in pairs (s, s + 1) on packed fp32 pairs: each pair accumulates two output
+    // blocks of one token in one FFMA2 per term.
     constexpr int HB = P / 2;
+    constexpr int G = NT / HB;
     constexpr int NP = (NS + 1) / 2;              // slot pairs (an odd last slot pairs with a zero slot)
+    const int w = threadIdx.x / HB, k = threadIdx.x % HB;
+    const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
     f2 acc_r[NP][TT], acc_i[NP][TT];
   #pragma unroll
     for (int u = 0; u < NP; ++u)
   #pragma unroll
       for (int t = 0; t < TT; ++t) acc_r[u][t] = acc_i[u][t] = f2_bc(0.0f);
 
-    // c_hat of the summed block j + 1 is loaded (through L2) while block j is
-    // contracted, so the L2 latency overlaps the FMA work.
-    float cr_n[2 * NP], ci_n[2 * NP];
     auto load_c = [&](int j, float (&cr)[2 * NP], float (&ci)[2 * NP]) {
   #pragma unroll
       for (int s = 0; s < 2 * NP; ++s) {
-        const int pi = threadIdx.x + NT * s;
-        const int ol = pi / HB, k = pi % HB;
+        const int ol = w + G * s;
         if (s < NS && ol < QI) {
           const int ob = o0 + ol;
           const float* crow = chat + (int64_t)(BWDX ? (j * q + ob) : (ob * q + j)) * P;
@@ -189,67 +189,77 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
       }
     };
     // no guard on the slot here: a slot beyond the CTA's blocks has c = 0 (load_c), so
-    // its accumulators stay 0 and are never stored; slots that share a bin (all of
-    // them when NT >= p/2) share the loads of X.
-    auto contract = [&](int j, const float (&cr_c)[2 * NP], const float (&ci_c)[2 * NP]) {
+    // its accumulators stay 0 and are never stored; all slots share the loads of X.
+    // The packed product as acc_r += cr xa + ci xb, acc_i += cr xc + ci xd, with the
+    // token's x terms chosen once for all slots:
+    //   forward, complex bin : xa = xr, xb = -xi, xc = xi, xd =  xr   (c x)
+    //   grad_x,  complex bin : xa = xr, xb =  xi, xc = xi, xd = -xr   (conj(c) x)
+    //   bin 0 (real pair)    : xa = xr, xb =   0, xc =  0, xd =  xi   (component-wise)
+    // bin0 = false (a warp with no bin-0 lane) drops the bin-0 selects.
+    auto contract = [&](bool bin0, int j, const float (&cr_c)[2 * NP], const float (&ci_c)[2 * NP]) {
+      f2 cr[NP], ci[NP];
+  #pragma unroll
+      for (int u = 0; u < NP; ++u) {
+        cr[u] = f2_mk(cr_c[2 * u], cr_c[2 * u + 1]);
+        ci[u] = f2_mk(ci_c[2 * u], ci_c[2 * u + 1]);
+      }
+      const bool z = bin0 && (k == 0);
   #pragma unroll
       for (int t = 0; t < TT; ++t) {
         const int rb = LayerGeo<P>::row_base(t * q + j);
+        const float vr = tile[rb + kr], vi = tile[rb + ki];
+        const f2 xa = f2_bc(vr);
+        const f2 xb = f2_bc(z ? 0.0f : (BWDX ? vi : -vi));
+        const f2 xc = f2_bc(z ? 0.0f : vi);
+        const f2 xd = f2_bc(z ? vi : (BWDX ? -vr : vr));
   #pragma unroll
         for (int u = 0; u < NP; ++u) {
-          const int k0 = (threadIdx.x + NT * (2 * u)) % HB, k1 = (threadIdx.x + NT * (2 * u + 1)) % HB;
-          // packed product: bin 0 multiplies the real pair component-wise, other bins are
-          // complex products (conjugated c for grad_x):
-          //   acc_r += cr xr + a2 xi,  acc_i += a3 xi + a4 xr
-          const float ci0 = ci_c[2 * u], ci1 = ci_c[2 * u + 1];
-          const bool z0 = (k0 == 0), z1 = (k1 == 0);
-          const f2 c1 = f2_mk(cr_c[2 * u], cr_c[2 * u + 1]);
-          const f2 c2 = f2_mk(z0 ? 0.0f : (BWDX ? ci0 : -ci0), z1 ? 0.0f : (BWDX ? ci1 : -ci1));
-          const f2 c3 = f2_mk(z0 ? ci0 : cr_c[2 * u], z1 ? ci1 : cr_c[2 * u + 1]);
-          const f2 c4 = f2_mk(z0 ? 0.0f : (BWDX ? -ci0 : ci0), z1 ? 0.0f : (BWDX ? -ci1 : ci1));
-          const f2 xr = f2_mk(tile[rb + LayerGeo<P>::at(k0)], tile[rb + LayerGeo<P>::at(k1)]);
-          const f2 xi = f2_mk(tile[rb + LayerGeo<P>::at(bin_im_slot<P>(k0))],
-                              tile[rb + LayerGeo<P>::at(bin_im_slot<P>(k1))]);
-          acc_r[u][t] = f2_fma(c1, xr, f2_fma(c2, xi, acc_r[u][t]));
-          acc_i[u][t] = f2_fma(c3, xi, f2_fma(c4, xr, acc_i[u][t]));
+          acc_r[u][t] = f2_fma(cr[u], xa, f2_fma(ci[u], xb, acc_r[u][t]));
+          acc_i[u][t] = f2_fma(cr[u], xc, f2_fma(ci[u], xd, acc_i[u][t]));
         }
       }
     };
     // a block's contraction is too short to hide an L2 round trip, so the c_hat of KB
     // summed blocks is requested at once (at most 32 floats), then contracted
     constexpr int KB = 8 / NP < 8 ? 8 / NP : 8;
-    if constexpr (KB > 1) {
-      for (int j0 = 0; j0 < q; j0 += KB) {
-        float crb[KB][2 * NP], cib[KB][2 * NP];
+    auto contract_all = [&](bool bin0) {
+      if constexpr (KB > 1) {
+        for (int j0 = 0; j0 < q; j0 += KB) {
+          float crb[KB][2 * NP], cib[KB][2 * NP];
   #pragma unroll
-        for (int d = 0; d < KB; ++d)
-          if (j0 + d < q) load_c(j0 + d, crb[d], cib[d]);
+          for (int d = 0; d < KB; ++d)
+            if (j0 + d < q) load_c(j0 + d, crb[d], cib[d]);
   #pragma unroll
-        for (int d = 0; d < KB; ++d)
-          if (j0 + d < q) contract(j0 + d, crb[d], cib[d]);
-      }
-    } else {
-      load_c(0, cr_n, ci_n);
-      for (int j = 0; j < q; ++j) {               // j: summed block (input j for fwd, output i for grad_x)
-        float cr_c[2 * NP], ci_c[2 * NP];
-  #pragma unroll
-        for (int sl = 0; sl < 2 * NP; ++sl) {
-          cr_c[sl] = cr_n[sl];
-          ci_c[sl] = ci_n[sl];
+          for (int d = 0; d < KB; ++d)
+            if (j0 + d < q) contract(bin0, j0 + d, crb[d], cib[d]);
         }
-        if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
-        contract(j, cr_c, ci_c);
+      } else {
+        // c_hat of the summed block j + 1 is loaded while block j is contracted
+        float cr_n[2 * NP], ci_n[2 * NP];
+        load_c(0, cr_n, ci_n);
+        for (int j = 0; j < q; ++j) {             // j: summed block (input j for fwd, output i for grad_x)
+          float cr_c[2 * NP], ci_c[2 * NP];
+  #pragma unroll
+          for (int sl = 0; sl < 2 * NP; ++sl) {
+            cr_c[sl] = cr_n[sl];
+            ci_c[sl] = ci_n[sl];
+          }
+          if (j + 1 < q) load_c(j + 1, cr_n, ci_n);
+          contract(bin0, j, cr_c, ci_c);
+        }
       }
-    }
+    };
+    // a warp holds bin 0 when its first lane does (p/2 >= 32); a warp-uniform branch, so
+    // each side is specialised
+    if ((threadIdx.x & ~31u) % HB == 0) contract_all(true);
+    else contract_all(false);
     __syncthreads();
 
     // 3. output spectra over the tile: row t*QI + ol
   #pragma unroll
     for (int s = 0; s < NS; ++s) {
-      const int pi = threadIdx.x + NT * s;
-      const int ol = pi / HB, k = pi % HB;
+      const int ol = w + G * s;
       if (ol < QI) {
-        const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
   #pragma unroll
         for (int t = 0; t < TT; ++t) {
           // stored mirrored (slot k = Re - Im, slot p-k = Re + Im) for the Hartley-form
@@ -423,48 +433,56 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
         return x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P;
       });
       __syncthreads();
-  #pragma unroll
-      for (int n = 0; n < NG; ++n) {
-        const int gam = threadIdx.x + NT * n;
-        if (gam < ngroups) {
-          const int k = gam % HB;
-          const int rest = gam / HB;
-          const int ib = rest % nib, jb = rest / nib;
-          const bool z = (k == 0);
-          const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
-          for (int t = 0; t < ntok; ++t) {
-            float gr[RI], gi[RI];
-  #pragma unroll
-            for (int a = 0; a < RI; ++a) {
-              const int rb = LayerGeo<P>::row_base(t * q + ib * RI + a);
-              gr[a] = tile[rb + kr];
-              gi[a] = tile[rb + ki];
-            }
-  #pragma unroll
-            for (int bp = 0; bp < RJP; ++bp) {
-              float xr[2], xi[2];
-  #pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                const int b = 2 * bp + h < RJ ? 2 * bp + h : RJ - 1;   // odd RJ: the spare half repeats b
-                const int rb = LayerGeo<P>::row_base(xrow0 + t * QJ + jb * RJ + b);
-                xr[h] = tile[rb + kr];
-                xi[h] = tile[rb + ki];
-              }
-              // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)
-              const f2 vxr = f2_mk(xr[0], xr[1]);
-              const f2 vxi_re = z ? f2_bc(0.0f) : f2_mk(xi[0], xi[1]);
-              const f2 vx_im = z ? f2_mk(xi[0], xi[1]) : f2_mk(xr[0], xr[1]);
-              const f2 vxi_im = z ? f2_bc(0.0f) : f2_mk(-xi[0], -xi[1]);
-  #pragma unroll
+      // bin0 = false (warps with no bin-0 group) drops the real-pair selects
+      auto accumulate = [&](bool bin0) {
+    #pragma unroll
+        for (int n = 0; n < NG; ++n) {
+          const int gam = threadIdx.x + NT * n;
+          if (gam < ngroups) {
+            const int k = gam % HB;
+            const int rest = gam / HB;
+            const int ib = rest % nib, jb = rest / nib;
+            const bool z = bin0 && (k == 0);
+            const int kr = LayerGeo<P>::at(k), ki = LayerGeo<P>::at(bin_im_slot<P>(k));
+            for (int t = 0; t < ntok; ++t) {
+              float gr[RI], gi[RI];
+    #pragma unroll
               for (int a = 0; a < RI; ++a) {
-                const f2 vgr = f2_bc(gr[a]), vgi = f2_bc(gi[a]);
-                s_r[n][a][bp] = f2_fma(vgr, vxr, f2_fma(vgi, vxi_re, s_r[n][a][bp]));
-                s_i[n][a][bp] = f2_fma(vgi, vx_im, f2_fma(vgr, vxi_im, s_i[n][a][bp]));
+                const int rb = LayerGeo<P>::row_base(t * q + ib * RI + a);
+                gr[a] = tile[rb + kr];
+                gi[a] = tile[rb + ki];
+              }
+    #pragma unroll
+              for (int bp = 0; bp < RJP; ++bp) {
+                float xr[2], xi[2];
+    #pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  const int b = 2 * bp + h < RJ ? 2 * bp + h : RJ - 1;   // odd RJ: the spare half repeats b
+                  const int rb = LayerGeo<P>::row_base(xrow0 + t * QJ + jb * RJ + b);
+                  xr[h] = tile[rb + kr];
+                  xi[h] = tile[rb + ki];
+                }
+                // G conj(X): re = gr xr + gi xi, im = gi xr - gr xi; bin 0: (gr xr, gi xi)
+                const f2 vxr = f2_mk(xr[0], xr[1]);
+                const f2 vxi_re = z ? f2_bc(0.0f) : f2_mk(xi[0], xi[1]);
+                const f2 vx_im = z ? f2_mk(xi[0], xi[1]) : f2_mk(xr[0], xr[1]);
+                const f2 vxi_im = z ? f2_bc(0.0f) : f2_mk(-xi[0], -xi[1]);
+    #pragma unroll
+                for (int a = 0; a < RI; ++a) {
+                  const f2 vgr = f2_bc(gr[a]), vgi = f2_bc(gi[a]);
+                  s_r[n][a][bp] = f2_fma(vgr, vxr, f2_fma(vgi, vxi_re, s_r[n][a][bp]));
+                  s_i[n][a][bp] = f2_fma(vgi, vx_im, f2_fma(vgr, vxi_im, s_i[n][a][bp]));
+                }
               }
             }
           }
         }
-      }
+      };
+      // a warp holds a bin-0 group only if its first lane does (gamma = tid + NT n with
+      // NT and p/2 multiples of 32, and p/2 a multiple of NT when larger); a warp-uniform
+      // branch, so each side is specialised
+      if ((threadIdx.x & ~31u) % HB == 0) accumulate(true);
+      else accumulate(false);
     }
     // add this CTA's partial packed cross-spectrum into grad_c
     griddep_launch_dependents();
