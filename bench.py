@@ -478,6 +478,46 @@ def run_layer_bench(rd, torch, dev, gen, hbm_peak, fp32_peak, n_sets_bytes=256 <
     return out, dominant
 
 
+def torch_fft_circulant(torch, x, c):
+    """y = W x of the block-circulant layer the usual way (a measured reference, not the
+    product): rfft of each block, per-bin complex contraction with rfft(c), irfft; fp32
+    compute, the output cast back to the input's dtype."""
+    B, D = x.shape
+    q, _, p = c.shape
+    xf = torch.fft.rfft(x.float().view(B, q, p), dim=-1)
+    cf = torch.fft.rfft(c, dim=-1)
+    yf = torch.einsum("ijk,bjk->bik", cf, xf)
+    return torch.fft.irfft(yf, n=p, dim=-1).reshape(B, D).to(x.dtype)
+
+
+def time_torch_fft_reference(torch, dev, gen, dt, B=256, D=4096, p=128, iters=50):
+    """Forward + backward time of torch_fft_circulant at one workload, for context beside
+    the layer's own numbers (eager launches, CUDA events, after warm-up)."""
+    q = D // p
+    c = (torch.randn(q, q, p, device=dev, generator=gen) / 64.0).requires_grad_(True)
+    x = torch.randn(B, D, device=dev, generator=gen).to(dt).requires_grad_(True)
+    g = torch.randn(B, D, device=dev, generator=gen).to(dt)
+
+    def step():
+        y = torch_fft_circulant(torch, x, c)
+        y.backward(g)
+
+    for _ in range(5):
+        step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(iters):
+        step()
+    b.record()
+    torch.cuda.synchronize()
+    us = a.elapsed_time(b) * 1e3 / iters
+    return {"fwd_bwd_us": round(us, 2), "tokens_s": round(B / (us * 1e-6), 1), "B": B, "D": D, "p": p,
+            "note": "torch.fft rfft/irfft + complex einsum, fp32 compute, bf16 activations, autograd backward; "
+                    "eager launches, context only"}
+
+
 def run_adapter_stack(rd, torch, dev, gen, world, max_over_ranks_, barrier):
     """LLaMA2-7B-shaped stack: 32 layers x (q, v) adapters of D = 4096, p = 512, 4096
     tokens per rank per step; every adapter's forward then every backward, grad_c of all
@@ -794,7 +834,25 @@ def run_ours(args):
                 key = f"B{Bm}_p{pm}_MB" + ("_inplace_spectrum" if inplace else "")
                 memory[key] = round((torch.cuda.max_memory_allocated(dev) - base) / 1e6, 3)
                 del lay, xm, ym
+    # the same training step for the usual FFT formulation, as a measured reference: torch
+    # (cuFFT) rfft / irfft of each block, the per-bin contraction as a complex einsum, fp32
+    # compute (cuFFT takes no bf16) with bf16 activations at the boundary; autograd keeps
+    # what it needs for the backward
+    for Bm in (1, 256):
+        for pm in (128, 512, 1024, 4096):
+            qm = 4096 // pm
+            torch.cuda.synchronize()
+            base = torch.cuda.memory_allocated(dev)
+            torch.cuda.reset_peak_memory_stats(dev)
+            cm = (torch.randn(qm, qm, pm, device=dev, generator=gen) / 64.0).requires_grad_(True)
+            xm = torch.randn(Bm, 4096, device=dev, generator=gen).to(dt).requires_grad_(True)
+            ym = torch_fft_circulant(torch, xm, cm)
+            ym.backward(torch.ones_like(ym))
+            torch.cuda.synchronize()
+            memory[f"torch_fft_B{Bm}_p{pm}_MB"] = round((torch.cuda.max_memory_allocated(dev) - base) / 1e6, 3)
+            del cm, xm, ym
     layer["single_layer_train_step_peak_memory_d4096_bf16"] = memory
+    layer["torch_fft_reference_d4096_p128_B256"] = time_torch_fft_reference(torch, dev, gen, dt)
 
     # ---- 2-D rdFFT and the explicit-spectrum cast (beside the step, not in it)
     spectral = {}

@@ -64,3 +64,21 @@ def test_clock_summary_reads_reasons():
 def statistics_median(v):
     import statistics
     return statistics.median(v)
+
+
+def test_torch_fft_reference_matches_the_oracle():
+    """The torch.fft circulant the bench measures for context computes the same layer as
+    the oracle's dense circulant (paper-notes page, "Circulant matrix training
+    adaptation"), so its memory and time figures describe the same work."""
+    import numpy as np
+    import torch
+
+    import oracle
+
+    gen = torch.Generator().manual_seed(11)
+    for q, p in ((1, 16), (4, 16), (3, 8)):
+        x = torch.randn(5, q * p, generator=gen)
+        c = torch.randn(q, q, p, generator=gen)
+        y = bench.torch_fft_circulant(torch, x, c).double().numpy()
+        ref = oracle.circ_forward(x.double().numpy(), c.double().numpy())
+        assert np.abs(y - ref).max() <= 1e-5 * np.abs(ref).max()
