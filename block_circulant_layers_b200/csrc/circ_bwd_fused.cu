@@ -30,7 +30,12 @@
 namespace rdfft {
 namespace {
 
-template <int P, int Q, typename T, int NT, int TT, int RI, int RJ>
+// QJ: the input blocks j of a CTA group (blockIdx.y): the CTA transforms g in full but x
+// only for its group's blocks, keeps the cross-spectrum S_ij of its group (every i) and
+// forms grad_x for its group's blocks. QJ = q for layers with few blocks; at q = 32 (p = 128)
+// four groups keep each CTA's part within tensor memory, and g is transformed once per group
+// (4 times a token, against 6 times for the separate grad_x and grad_c kernels).
+template <int P, int Q, int QJ, typename T, int NT, int TT, int RI, int RJ>
 __global__ void __launch_bounds__(NT, 1)
 k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* __restrict__ chat,
                  T* __restrict__ grad_x, float* __restrict__ grad_c, int64_t B, int64_t tok_per_cta) {
@@ -39,14 +44,18 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
   constexpr int HB = P / 2;
   constexpr int RJP = RJ / 2;
   constexpr int ACC = RI * RJ * 2;                  // floats of cross-spectrum per thread
-  constexpr int NS = Q * HB / NT;                   // grad_x output blocks per thread (one bin)
-  constexpr int CH = NS * Q * 2;                    // floats of c_hat per thread
+  constexpr int NS = QJ * HB / NT;                  // grad_x output blocks per thread (one bin)
+  constexpr int CPI = 2 * NS;                       // c_hat floats per thread and summed block i
+  constexpr int BPL = 16 / CPI;                     // summed blocks per 16-column tensor-memory load
+  constexpr int CH = CPI * Q;                       // floats of c_hat per thread
   constexpr int PER = ACC + CH;                     // tensor-memory columns per thread
   constexpr int WQ = NT / 128;                      // warps per tensor-memory lane quarter
   constexpr int COLS = WQ * PER;
   static_assert(RJ % 2 == 0 && ACC % 16 == 0 && CH % 16 == 0, "accumulator layout");
   static_assert((COLS & (COLS - 1)) == 0 && COLS >= 32 && COLS <= 512, "tensor-memory allocation");
   static_assert(NT % HB == 0 && NS >= 1, "the grad_x slots of a thread share one bin");
+  static_assert(Q % QJ == 0 && QJ % RJ == 0 && 16 % CPI == 0 && Q % BPL == 0, "block groups");
+  static_assert(NS % 2 == 0 || (NS == 1 && TT % 2 == 0), "slot pairs, or token pairs for one slot");
   extern __shared__ float tile[];
   __shared__ uint32_t tmem_holder;
   const int D = q * P;
@@ -54,9 +63,10 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
   const int64_t tend = (tbeg + tok_per_cta < B) ? tbeg + tok_per_cta : B;
   const bool sole = (gridDim.x == 1);
   const int warp = threadIdx.x >> 5;
+  const int j0 = blockIdx.y * QJ;                   // the group's first input block
   const int nib = q / RI;
-  const int ng = HB * nib * (q / RJ);               // cross-spectrum groups (one per thread)
-  const int XR = TT * q;                            // first X row of the tile
+  const int ng = HB * nib * (QJ / RJ);              // cross-spectrum groups (one per thread)
+  const int XR = TT * q;                            // first X row of the tile (a multiple of 32)
 
   griddep_wait();
   if (warp == 0) tc::tmem_alloc(&tmem_holder, COLS);
@@ -71,18 +81,18 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
 #pragma unroll
   for (int c = 0; c < ACC; c += 16) tc::tmem_st16(tacc + c, acc + c);
 
-  // the thread's cross-spectrum group: bin k, output blocks ib*RI.., input blocks jb*RJ..
+  // the thread's cross-spectrum group: bin k, output blocks ib*RI.., input blocks j0 + jb*RJ..
   const int gam = threadIdx.x;
   const int gk = gam % HB, gib = (gam / HB) % nib, gjb = gam / HB / nib;
   // a warp holds bin 0 (grad_c group or grad_x slot) only if its first lane does; such
   // warps take the real pair's component-wise products, the others the complex ones
   const bool warp_bin0 = (threadIdx.x & ~31u) % HB == 0;
   const int gkr = G::at(gk), gki = G::at(bin_im_slot<P>(gk));
-  // the thread's grad_x slots: bin xk, output blocks o_u = xo0 + u NT / HB (u < NS). Their
-  // c_hat values (for every summed block i) are the same for every token: read once here
-  // and kept in tensor memory beside the cross-spectrum, as [i][slot pair w] (re_2w,
-  // re_2w+1, im_2w, im_2w+1) (16 columns = two summed blocks), with conj(c_hat) and bin 0's
-  // real pair applied at use.
+  // the thread's grad_x slots: bin xk, output blocks j0 + o_u, o_u = xo0 + u NT / HB (u < NS).
+  // Their c_hat values (for every summed block i) are the same for every token: read once
+  // here and kept in tensor memory beside the cross-spectrum, as [i][slot pair w] (re_2w,
+  // re_2w+1, im_2w, im_2w+1), or [i] (re, im) for a single slot (16 columns = BPL summed
+  // blocks), with conj(c_hat) and bin 0's real pair applied at use.
   constexpr int XG = NT / HB;
   const int xk = threadIdx.x % HB, xo0 = threadIdx.x / HB;
   const int xkr = G::at(xk), xki = G::at(bin_im_slot<P>(xk));
@@ -92,10 +102,10 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
     for (int u = 0; u < NS; ++u)
 #pragma unroll
       for (int i = 0; i < Q; ++i) {
-        const float* crow = chat + (int64_t)(i * Q + xo0 + u * XG) * P;
-        const int c = 2 * (i * NS + (u & ~1)) + (u & 1);
+        const float* crow = chat + (int64_t)(i * Q + j0 + xo0 + u * XG) * P;
+        const int c = NS == 1 ? CPI * i : CPI * i + 2 * (u & ~1) + (u & 1);
         ch[c] = __ldg(crow + xk);
-        ch[c + 2] = __ldg(crow + bin_im_slot<P>(xk));
+        ch[c + (NS == 1 ? 1 : 2)] = __ldg(crow + bin_im_slot<P>(xk));
       }
 #pragma unroll
     for (int c = 0; c < CH; c += 16) tc::tmem_st16(tch + c, ch + c);
@@ -105,13 +115,14 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
   for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
     const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
     if (tok0 != tbeg) __syncthreads();              // the previous tile is fully consumed
-    // 1. rdFFT of g (rows t q + i) and x (rows XR + t q + j) of the tile's tokens
-    fft_rows<P, NT, T>(tile, 2 * XR, [&](int r) -> const T* {
-      const bool isx = r >= XR;
-      const int rr = isx ? r - XR : r;
-      const int t = rr / q, b = rr - t * q;
-      if (t >= ntok) return nullptr;
-      return (isx ? x : g) + (tok0 + t) * (int64_t)D + (int64_t)b * P;
+    // 1. rdFFT of g (rows t q + i) and of the group's x blocks (rows XR + t QJ + jl)
+    fft_rows<P, NT, T>(tile, XR + TT * QJ, [&](int r) -> const T* {
+      if (r < XR) {
+        const int t = r / q, b = r - t * q;
+        return t < ntok ? g + (tok0 + t) * (int64_t)D + (int64_t)b * P : nullptr;
+      }
+      const int t = (r - XR) / QJ, jl = r - XR - t * QJ;
+      return t < ntok ? x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
     });
     __syncthreads();
 
@@ -138,7 +149,7 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
           float xr[2], xi[2];
 #pragma unroll
           for (int h = 0; h < 2; ++h) {
-            const int rb = G::row_base(XR + t * q + gjb * RJ + 2 * bp + h);
+            const int rb = G::row_base(XR + t * QJ + gjb * RJ + 2 * bp + h);
             xr[h] = tile[rb + gkr];
             xi[h] = tile[rb + gki];
           }
@@ -171,27 +182,26 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
 
     // 3. grad_x spectra over the X rows: Y_j = sum_i conj(C_ij) G_i, stored mirrored
     // (slot k = Re - Im, slot p - k = Re + Im; bin 0 keeps its real pair)
-    {
+    // conj(c) G as yr += cr xa + ci xb, yi += cr xc + ci xd with the token's G terms
+    //   complex bin: xa = gr, xb = gi, xc = gi, xd = -gr;  bin 0: xa = gr, xb = xc = 0, xd = gi
+    if constexpr (NS % 2 == 0) {
       // all NS slots share the bin, so each G value is read once for all of them; slot
       // pairs (u, u + 1) accumulate on packed fp32 pairs
-      static_assert(NS % 2 == 0 && 2 * NS == 8 && Q % 2 == 0, "slot pairs; two summed blocks per 16 columns");
       f2 yr[NS / 2][TT], yi[NS / 2][TT];
 #pragma unroll
       for (int w = 0; w < NS / 2; ++w)
 #pragma unroll
         for (int t = 0; t < TT; ++t) yr[w][t] = yi[w][t] = f2_bc(0.0f);
-      // conj(c) G as yr += cr xa + ci xb, yi += cr xc + ci xd with the token's G terms
-      //   complex bin: xa = gr, xb = gi, xc = gi, xd = -gr;  bin 0: xa = gr, xb = xc = 0, xd = gi
       auto contract = [&](bool bin0) {
         const bool xz = bin0 && (xk == 0);
         float ch[16];
 #pragma unroll
         for (int i = 0; i < Q; ++i) {
-          if ((i & 1) == 0) {
-            tc::tmem_ld16_nowait(tch + 2 * i * NS, ch);
+          if (i % BPL == 0) {
+            tc::tmem_ld16_nowait(tch + CPI * i, ch);
             tc::tmem_wait_ld();
           }
-          const int cb = 2 * (i & 1) * NS;
+          const int cb = CPI * (i % BPL);
           f2 cr[NS / 2], ci[NS / 2];
 #pragma unroll
           for (int w = 0; w < NS / 2; ++w) {
@@ -226,18 +236,60 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
           if (t < ntok) {
             const float ar = (u & 1) ? yr[u / 2][t].y : yr[u / 2][t].x;
             const float ai = (u & 1) ? yi[u / 2][t].y : yi[u / 2][t].x;
-            const int rb = G::row_base(XR + t * Q + o);
+            const int rb = G::row_base(XR + t * QJ + o);
             tile[rb + xkr] = xk == 0 ? ar : ar - ai;
             tile[rb + xki] = xk == 0 ? ai : ar + ai;
           }
         }
       }
+    } else {
+      // one slot: token pairs (t, t + 1) accumulate on packed fp32 pairs, c_hat broadcast
+      f2 yr[TT / 2], yi[TT / 2];
+#pragma unroll
+      for (int v = 0; v < TT / 2; ++v) yr[v] = yi[v] = f2_bc(0.0f);
+      auto contract = [&](bool bin0) {
+        const bool xz = bin0 && (xk == 0);
+        float ch[16];
+#pragma unroll
+        for (int i = 0; i < Q; ++i) {
+          if (i % BPL == 0) {
+            tc::tmem_ld16_nowait(tch + CPI * i, ch);
+            tc::tmem_wait_ld();
+          }
+          const int cb = CPI * (i % BPL);
+          const f2 cr = f2_bc(ch[cb]), ci = f2_bc(ch[cb + 1]);
+#pragma unroll
+          for (int v = 0; v < TT / 2; ++v) {
+            // rows of tokens beyond ntok hold zeros (their transforms read no input)
+            const int rb0 = G::row_base(2 * v * Q + i), rb1 = G::row_base((2 * v + 1) * Q + i);
+            const float vr0 = tile[rb0 + xkr], vi0 = tile[rb0 + xki];
+            const float vr1 = tile[rb1 + xkr], vi1 = tile[rb1 + xki];
+            const f2 xa = f2_mk(vr0, vr1);
+            const f2 xb = xz ? f2_bc(0.0f) : f2_mk(vi0, vi1);
+            const f2 xd = xz ? f2_mk(vi0, vi1) : f2_mk(-vr0, -vr1);
+            yr[v] = f2_fma(cr, xa, f2_fma(ci, xb, yr[v]));
+            yi[v] = f2_fma(cr, xb, f2_fma(ci, xd, yi[v]));
+          }
+        }
+      };
+      if (warp_bin0) contract(true);                 // warp-uniform: each side is specialised
+      else contract(false);
+#pragma unroll
+      for (int t = 0; t < TT; ++t) {
+        if (t < ntok) {
+          const float ar = (t & 1) ? yr[t / 2].y : yr[t / 2].x;
+          const float ai = (t & 1) ? yi[t / 2].y : yi[t / 2].x;
+          const int rb = G::row_base(XR + t * QJ + xo0);
+          tile[rb + xkr] = xk == 0 ? ar : ar - ai;
+          tile[rb + xki] = xk == 0 ? ai : ar + ai;
+        }
+      }
     }
     __syncthreads();
     // 4. rdIFFT (Hartley form) of the grad_x rows straight to HBM
-    ifft_rows_mirrored<P, NT, T>(tile + G::row_base(XR), XR, [&](int r) -> T* {
-      const int t = r / q, j = r - t * q;
-      return t < ntok ? grad_x + (tok0 + t) * (int64_t)D + (int64_t)j * P : nullptr;
+    ifft_rows_mirrored<P, NT, T>(tile + G::row_base(XR), TT * QJ, [&](int r) -> T* {
+      const int t = r / QJ, jl = r - t * QJ;
+      return t < ntok ? grad_x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
     });
   }
 
@@ -252,7 +304,7 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
     for (int a = 0; a < RI; ++a)
 #pragma unroll
       for (int b = 0; b < RJ; ++b) {
-        float* dst = grad_c + ((int64_t)(gib * RI + a) * q + (gjb * RJ + b)) * P;
+        float* dst = grad_c + ((int64_t)(gib * RI + a) * q + (j0 + gjb * RJ + b)) * P;
         const int o = (a * RJP + b / 2) * 4 + (b & 1);
         const float vr = acc[o], vi = acc[o + 2];
         if (sole) {
@@ -269,36 +321,42 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
   if (warp == 0) tc::tmem_dealloc(tmem_holder, COLS);
 }
 
-template <int P, int Q, typename T, int TT, int RI, int RJ>
+template <int P, int Q, int QJ, typename T, int TT, int RI, int RJ>
 cudaError_t run_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B,
                       cudaStream_t s) {
   constexpr int NT = 512;
   constexpr int q = Q;
-  auto kern = k_circ_bwd_fused<P, Q, T, NT, TT, RI, RJ>;
-  const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(2 * TT * q);
+  auto kern = k_circ_bwd_fused<P, Q, QJ, T, NT, TT, RI, RJ>;
+  const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(TT * (q + QJ));
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
+  constexpr int NJG = Q / QJ;                      // input-block groups
   int64_t tiles_per = 1;
-  const int slices = layer_gc_slices(1, (B + TT - 1) / TT, num_sms(), &tiles_per);
+  const int slices = layer_gc_slices(NJG, (B + TT - 1) / TT, num_sms(), &tiles_per);
   if (slices > 1) {
     e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)q * q * P, s);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(kern, dim3((unsigned)slices), dim3(NT), smem, s, static_cast<const T*>(g),
+  return launch_pdl(kern, dim3((unsigned)slices, (unsigned)NJG), dim3(NT), smem, s, static_cast<const T*>(g),
                     static_cast<const T*>(x), chat, static_cast<T*>(grad_x), grad_c, B, (int64_t)(tiles_per * TT));
 }
 
 template <typename T>
 cudaError_t fused_t(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B, int q,
                     int p, cudaStream_t s) {
-  if (p == 512 && q == 8) return run_fused<512, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s);
-  if (p == 1024 && q == 4) return run_fused<1024, 4, T, 2, 4, 4>(g, x, chat, grad_x, grad_c, B, s);
+  if (p == 128 && q == 32) return run_fused<128, 32, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s);
+  if (p == 512 && q == 8) return run_fused<512, 8, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s);
+  if (p == 1024 && q == 4) return run_fused<1024, 4, 4, T, 2, 4, 4>(g, x, chat, grad_x, grad_c, B, s);
   return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
-bool circ_bwd_fused_supported(int p, int D) { return (p == 512 && D == 4096) || (p == 1024 && D == 4096); }
+// p = 128 (q = 32) from 256 tokens on: its tiles always hold TT tokens' rows, so small
+// batches stay with the two kernels, whose grids adapt to a handful of tokens
+bool circ_bwd_fused_supported(int p, int D, int64_t B) {
+  return (p == 512 && D == 4096) || (p == 1024 && D == 4096) || (p == 128 && D == 4096 && B >= 256);
+}
 
 cudaError_t launch_circ_bwd_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c,
                                   int64_t B, int D, int p, int dtype, cudaStream_t s) {

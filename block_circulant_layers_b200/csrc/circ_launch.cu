@@ -36,7 +36,7 @@ cudaError_t launch_circ_bwd(const void* g, const void* x, const float* c_hat, vo
                             float* grad_c, int64_t B, int D, int p, int dtype, cudaStream_t s) {
   const int q = D / p;
   cudaError_t e = cudaSuccess;
-  if (grad_c != nullptr && grad_x != nullptr && circ_bwd_fused_supported(p, D)) {
+  if (grad_c != nullptr && grad_x != nullptr && circ_bwd_fused_supported(p, D, B)) {
     // both gradients from one transform of g and x (circ_bwd_fused.cu), then grad_c's rdIFFT
     e = launch_circ_bwd_fused(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, s);
     if (e == cudaSuccess) e = launch_rows(grad_c, (int64_t)q * q, p, 0, true, s);

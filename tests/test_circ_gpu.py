@@ -101,6 +101,15 @@ def test_fused_backward_shapes(rd, p, B, dtype):
     check_all(rd, B, 4096, p, dtype, (110 + p, 120 + B, 130 + B))
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B", [256, 259, 301])
+def test_fused_backward_p128_block_groups(rd, B, dtype):
+    """D = 4096 at p = 128 (q = 32) from 256 tokens: the fused backward splits the input
+    blocks into 4 groups (grid y), each CTA transforming g in full and x for its group, with
+    a ragged last token tile and several token slices adding into grad_c."""
+    check_all(rd, B, 4096, 128, dtype, (150, 151 + B, 152 + B))
+
+
 @pytest.mark.parametrize("p", [512, 1024])
 def test_fused_backward_stores_every_grad_c_element(rd, p):
     """With a single CTA (few tokens) the fused kernel stores grad_c instead of adding into a
