@@ -138,7 +138,8 @@ __device__ __forceinline__ int bin_im_slot(int k) { return k == 0 ? P / 2 : P - 
 // BWDX = true : in = g, out = grad_x; the CTA's QI output blocks are j, summed over i,
 //               against conj(c_hat).
 template <int P, typename T, int NT, int TT, int NS, bool BWDX>
-__global__ void __launch_bounds__(NT, NT >= 256 ? 2 : 1)   // 256-thread CTAs: two per SM (<= 128 registers)
+// 256-thread CTAs are declared for two per SM (<= 128 registers), 512-thread ones for one
+__global__ void __launch_bounds__(NT, NT >= 512 ? 1 : (NT >= 256 ? 2 : 1))
 k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict__ out,
          int64_t B, int q, int QI) {
   extern __shared__ float tile[];
@@ -643,11 +644,14 @@ static cudaError_t launch_x_p(const void* in, const float* chat, void* out, int6
                               cudaStream_t s) {
   if constexpr (P <= 512) {
     constexpr int NT = 256;
-    // up to 8 output blocks per CTA; 16 at p = 128 from B = 256 on, where fewer CTA
-    // groups transforming the same input rows pays (7% faster at D = 4096, B = 256; at
-    // B = 1 the 8-block CTAs, more of them, are 11% faster)
+    // up to 8 output blocks per CTA; at p = 128 from B = 256 on, 16 (fewer CTA groups
+    // transforming the same input rows: 7% faster at D = 4096, B = 256), and with q >= 16
+    // CTAs of 512 threads over 2 tokens and up to 32 output blocks, so each input row is
+    // transformed once (18.3 against 19.3 us at D = 4096, B = 256); at B = 1 the 8-block
+    // CTAs, more of them, are 11% faster
     constexpr int NS = (8 * (P / 2)) / NT > 0 ? (8 * (P / 2)) / NT : 1;
     if constexpr (P == 128) {
+      if (B >= 256 && q >= 16) return launch_x_cfg<P, T, 512, 2, 4, BWDX>(in, chat, out, B, q, s);
       if (B >= 256) return launch_x_cfg<P, T, NT, 4, 2 * NS, BWDX>(in, chat, out, B, q, s);
     }
     if (B >= 256 && NS * 4 <= 32) return launch_x_cfg<P, T, NT, 4, NS, BWDX>(in, chat, out, B, q, s);
