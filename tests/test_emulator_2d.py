@@ -63,3 +63,22 @@ def test_2d_unsupported_and_empty(emu):
     a = np.zeros((4, 6), dtype=np.float32)
     assert emu.rdfft2_emulate(a.ctypes.data, 1, 4, 6, 0, 0) == 1
     assert emu.rdfft2_emulate(None, 0, 64, 64, 0, 0) == 0
+
+
+@pytest.mark.parametrize("C", [32, 64])
+@pytest.mark.parametrize("inverse", [0, 1])
+def test_2d_bf16_r4096_interior_strips(emu, C, inverse):
+    """R = 4096, 16-bit, with interior strip pairs (away from columns 0 and C/2) as well as
+    the edge ones, forward and inverse against the oracle: a strip's left columns and their
+    mirrors land in the right tile rows and come back to the right image columns."""
+    s = sample(9100 + C + inverse, (1, 4096, C), "bf16")
+    a = s.stored.copy()
+    assert emu.rdfft2_emulate(a.ctypes.data, 1, 4096, C, 1, inverse) == 0
+    ref = (oracle.idft2_packed if inverse else oracle.dft2_packed)(s.exact)
+    got = bf16_bits_to_f64(a)
+    assert np.all(np.abs(got - ref) <= 2e-2 * np.sqrt(np.mean(ref ** 2)))
+    # every column pair is right, not just most of the image: the worst column's error
+    # stays at bf16 rounding size relative to that column's own scale
+    col_err = np.abs(got - ref).max(axis=(0, 1))
+    col_rms = np.sqrt(np.mean(ref ** 2, axis=(0, 1)))
+    assert np.all(col_err <= 2e-2 * np.maximum(col_rms, 1e-30) + 1e-6 * np.sqrt(np.mean(ref ** 2)))
