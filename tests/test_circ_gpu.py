@@ -178,6 +178,15 @@ def test_tensor_core_shape_rules(rd):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,D", [(256, 2048), (257, 8192), (256, 1024)])
+def test_p128_many_token_shapes(rd, B, D, dtype):
+    """p = 128 from 256 tokens with q = 16, 64 and 8: the 512-thread forward / grad_x CTAs
+    cover 16 output blocks (q = 16), two groups of 32 (q = 64, one token left over), or keep
+    the 256-thread shape (q < 16); the backward runs the two kernels (D != 4096)."""
+    check_all(rd, B, D, 128, dtype, (160, 161 + D // 128, 162 + B))
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("D,p,seed", [(4096, 1024, 7), (4096, 4096, 8), (1024, 1024, 9)])
 def test_config_block_size_extremes(rd, D, p, seed, dtype):
     check_all(rd, 256, D, p, dtype, (seed, seed + 10, seed + 20))
