@@ -352,10 +352,11 @@ cudaError_t fused_t(const void* g, const void* x, const float* chat, void* grad_
 
 }  // namespace
 
-// p = 128 (q = 32) from 256 tokens on: its tiles always hold TT tokens' rows, so small
-// batches stay with the two kernels, whose grids adapt to a handful of tokens
+// p = 128 (q = 32) from 64 tokens on (backward at D = 4096: 22.9 against 26.1 us at B = 64,
+// 25.0 against 31.8 at B = 128); below, the two kernels, whose grids adapt to a handful of
+// tokens, are faster (17.9 against 19.6 us at B = 1)
 bool circ_bwd_fused_supported(int p, int D, int64_t B) {
-  return (p == 512 && D == 4096) || (p == 1024 && D == 4096) || (p == 128 && D == 4096 && B >= 256);
+  return (p == 512 && D == 4096) || (p == 1024 && D == 4096) || (p == 128 && D == 4096 && B >= 64);
 }
 
 cudaError_t launch_circ_bwd_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c,

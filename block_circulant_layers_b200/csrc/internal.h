@@ -37,7 +37,7 @@ cudaError_t take_tc_device_error(unsigned int* flags);
 
 // Backward in one kernel (grad_x and the grad_c cross-spectrum from one transform of g
 // and x per input-block group) for the shapes it covers (circ_bwd_fused_supported: D = 4096
-// at p = 512 or 1024, and at p = 128 from B = 256); the caller runs the in-place rdIFFT of
+// at p = 512 or 1024, and at p = 128 from B = 64); the caller runs the in-place rdIFFT of
 // grad_c after it.
 bool circ_bwd_fused_supported(int p, int D, int64_t B);
 cudaError_t launch_circ_bwd_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c,

@@ -102,9 +102,9 @@ def test_fused_backward_shapes(rd, p, B, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("B", [256, 259, 301])
+@pytest.mark.parametrize("B", [64, 77, 256, 259, 301])
 def test_fused_backward_p128_block_groups(rd, B, dtype):
-    """D = 4096 at p = 128 (q = 32) from 256 tokens: the fused backward splits the input
+    """D = 4096 at p = 128 (q = 32) from 64 tokens: the fused backward splits the input
     blocks into 4 groups (grid y), each CTA transforming g in full and x for its group, with
     a ragged last token tile and several token slices adding into grad_c."""
     check_all(rd, B, 4096, 128, dtype, (150, 151 + B, 152 + B))
