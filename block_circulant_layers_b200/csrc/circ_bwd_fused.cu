@@ -1,5 +1,6 @@
-// Block-circulant layer backward in one kernel for layers with few blocks (q <= 8):
-// grad_x and grad_c from one transform of each token's g and x.
+// Block-circulant layer backward in one kernel: grad_x and grad_c from one transform of
+// each token's g and x per group of input blocks (one group for layers with few blocks,
+// q <= 8; four at q = 32).
 //
 // "Memory-Efficient Training with In-Place FFT Implementation", paper-notes page,
 // "Circulant matrix training adaptation" (gradients keep the conjugate symmetry):
@@ -18,9 +19,9 @@
 // accumulation of each tile, it leaves the registers to the transforms and the grad_x
 // contraction. Beside it each thread keeps the c_hat values of its grad_x slots (one
 // bin, NS output blocks, all q summed blocks: 64 floats at p = 512), read from HBM once
-// per CTA instead of once per tile. At the end each CTA adds its part into grad_c (fp32 red.add into a
-// zeroed grad_c; a plain store when one CTA covers all tokens), and the caller's
-// stream runs the in-place rdIFFT of grad_c's q^2 rows after, as circ_bwd does.
+// per CTA instead of once per tile. At the end each CTA adds its part into grad_c (fp32
+// red.add into a zeroed grad_c; a plain store when one CTA per group covers all tokens), and
+// the caller's stream runs the in-place rdIFFT of grad_c's q^2 rows after, as circ_bwd does.
 #include <cuda_runtime.h>
 
 #include "circ_kernels.cuh"

@@ -22,6 +22,8 @@
 //    into grad_c once (fp32 red.add; a plain store when a single token slice covers
 //    all tokens, and grad_c then needs no zeroing). grad_c is rdIFFT'd in place
 //    after, so the output buffer is the only global storage used.
+//  * For some shapes circ_bwd with both gradients runs one kernel instead of k_circ_x
+//    (grad_x) and k_circ_gc (circ_bwd_fused.cu).
 #pragma once
 
 #include <cuda_runtime.h>
