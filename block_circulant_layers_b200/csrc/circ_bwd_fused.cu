@@ -24,12 +24,31 @@
 // the caller's stream runs the in-place rdIFFT of grad_c's q^2 rows after, as circ_bwd does.
 #include <cuda_runtime.h>
 
+#include "bulk_copy.cuh"
 #include "circ_kernels.cuh"
 #include "internal.h"
 #include "tcgen05.cuh"
 
 namespace rdfft {
 namespace {
+
+#ifndef RDFFT_FUSED_STAGING
+#define RDFFT_FUSED_STAGING 1
+#endif
+
+// Shared memory of the fused kernel: the fp32 tile of TT (q + QJ) rows; with staging (16-bit
+// rows, p >= 512, where a warp's lanes span at most two rows of the staged tile) a buffer of
+// the next tile's g and x rows as they are in HBM, filled by bulk copies (the TMA engine, no
+// cluster multicast) while the current tile is processed, and its mbarrier.
+template <int P, int Q, int QJ, typename T, int TT>
+struct FusedSmem {
+  static constexpr bool STG = RDFFT_FUSED_STAGING && sizeof(T) == 2 && P >= 512;
+  static constexpr int TILE_WORDS = ((LayerGeo<P>::words(TT * (Q + QJ)) + 3) / 4) * 4;
+  static constexpr int STAGE_G = TT * Q * P;                     // elements: TT tokens' g rows
+  static constexpr int STAGE = STAGE_G + TT * QJ * P;            // and their x rows of the group
+  static constexpr size_t MBAR_OFF = sizeof(float) * (size_t)TILE_WORDS + (STG ? ((sizeof(T) * STAGE + 15) / 16) * 16 : 0);
+  static constexpr size_t BYTES = MBAR_OFF + (STG ? 16 : 0);
+};
 
 // QJ: the input blocks j of a CTA group (blockIdx.y): the CTA transforms g in full but x
 // only for its group's blocks, keeps the cross-spectrum S_ij of its group (every i) and
@@ -68,8 +87,27 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
   const int nib = q / RI;
   const int ng = HB * nib * (QJ / RJ);              // cross-spectrum groups (one per thread)
   const int XR = TT * q;                            // first X row of the tile (a multiple of 32)
+  using SM = FusedSmem<P, Q, QJ, T, TT>;
+  T* stage = reinterpret_cast<T*>(tile + SM::TILE_WORDS);
+  uint64_t* mbar = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(tile) + SM::MBAR_OFF);
+  // the rows of the tile starting at token tk into the staging buffer (thread 0)
+  auto fill = [&](int64_t tk) {
+    const int nt = (int)((tend - tk) < TT ? (tend - tk) : TT);
+    mbar_arrive_expect_tx(mbar, (unsigned)(nt * (D + QJ * P) * (int)sizeof(T)));
+    for (int t = 0; t < nt; ++t) {
+      bulk_load(stage + (size_t)t * D, g + (tk + t) * (int64_t)D, (unsigned)(D * sizeof(T)), mbar);
+      bulk_load(stage + SM::STAGE_G + (size_t)t * QJ * P, x + (tk + t) * (int64_t)D + (int64_t)j0 * P,
+                (unsigned)(QJ * P * sizeof(T)), mbar);
+    }
+  };
 
   griddep_wait();
+  if constexpr (SM::STG) {
+    if (threadIdx.x == 0) {
+      mbar_init(mbar, 1);
+      if (tbeg < tend) fill(tbeg);
+    }
+  }
   if (warp == 0) tc::tmem_alloc(&tmem_holder, COLS);
   tc::fence_before_sync();
   __syncthreads();
@@ -113,18 +151,46 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
   }
   tc::tmem_wait_st();
 
+  bool failed = false;
+  unsigned phase = 0;
   for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
     const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
     if (tok0 != tbeg) __syncthreads();              // the previous tile is fully consumed
-    // 1. rdFFT of g (rows t q + i) and of the group's x blocks (rows XR + t QJ + jl)
-    fft_rows<P, NT, T>(tile, XR + TT * QJ, [&](int r) -> const T* {
+    if constexpr (SM::STG) {                        // this tile's rows have landed (bounded wait)
+      const bool arrived = mbar_wait_bounded(mbar, phase);
+      phase ^= 1u;
+      if (!__syncthreads_and(arrived)) {
+        if (threadIdx.x == 0) mbar_wait_bounded(mbar, phase ^ 1u, kWaitCycles / 8);   // copies in flight
+        failed = true;
+        break;
+      }
+    }
+    // 1. rdFFT of g (rows t q + i) and of the group's x blocks (rows XR + t QJ + jl), read
+    // from the staging buffer or from HBM
+    auto src = [&](int r) -> const T* {
       if (r < XR) {
         const int t = r / q, b = r - t * q;
-        return t < ntok ? g + (tok0 + t) * (int64_t)D + (int64_t)b * P : nullptr;
+        if (t >= ntok) return nullptr;
+        return SM::STG ? stage + (size_t)t * D + (size_t)b * P : g + (tok0 + t) * (int64_t)D + (int64_t)b * P;
       }
       const int t = (r - XR) / QJ, jl = r - XR - t * QJ;
-      return t < ntok ? x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
-    });
+      if (t >= ntok) return nullptr;
+      return SM::STG ? stage + SM::STAGE_G + (size_t)(t * QJ + jl) * P
+                     : x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P;
+    };
+    {
+      constexpr int TPR = G::TPR, RPR = NT / TPR;
+      const int v = threadIdx.x % TPR;
+      for (int r = threadIdx.x / TPR; r < XR + TT * QJ; r += RPR) {
+        const T* row = src(r);
+        fwd_pass0<G, T>(tile, r, v, row, row != nullptr);
+      }
+    }
+    if constexpr (SM::STG) {
+      __syncthreads();                               // the staged rows are read: fetch the next tile's
+      if (threadIdx.x == 0 && tok0 + TT < tend) fill(tok0 + TT);
+    }
+    fft_rows_rest<P, NT, T, 1>(tile, XR + TT * QJ, src);
     __syncthreads();
 
     // 2. cross-spectrum: S_ij += G_i conj(X_j) over the tile's tokens, from and back to
@@ -294,12 +360,12 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
     });
   }
 
-  // 5. the CTA's cross-spectrum into grad_c
+  // 5. the CTA's cross-spectrum into grad_c (left unwritten after a wait gave up)
   griddep_launch_dependents();
 #pragma unroll
   for (int c = 0; c < ACC; c += 16) tc::tmem_ld16_nowait(tacc + c, acc + c);
   tc::tmem_wait_ld();
-  if (gam < ng) {
+  if (gam < ng && !failed) {
     const int kim = bin_im_slot<P>(gk);
 #pragma unroll
     for (int a = 0; a < RI; ++a)
@@ -328,7 +394,7 @@ cudaError_t run_fused(const void* g, const void* x, const float* chat, void* gra
   constexpr int NT = 512;
   constexpr int q = Q;
   auto kern = k_circ_bwd_fused<P, Q, QJ, T, NT, TT, RI, RJ>;
-  const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(TT * (q + QJ));
+  const size_t smem = FusedSmem<P, Q, QJ, T, TT>::BYTES;
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
   constexpr int NJG = Q / QJ;                      // input-block groups
@@ -356,6 +422,14 @@ cudaError_t fused_t(const void* g, const void* x, const float* chat, void* grad_
 // p = 128 (q = 32) from 64 tokens on (backward at D = 4096: 22.9 against 26.1 us at B = 64,
 // 25.0 against 31.8 at B = 128); below, the two kernels, whose grids adapt to a handful of
 // tokens, are faster (17.9 against 19.6 us at B = 1)
+cudaError_t take_fused_device_error(unsigned int* flags) {
+  unsigned int v = 0, zero = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+  *flags = v;
+  return e;
+}
+
 bool circ_bwd_fused_supported(int p, int D, int64_t B) {
   return (p == 512 && D == 4096) || (p == 1024 && D == 4096) || (p == 128 && D == 4096 && B >= 64);
 }

@@ -40,6 +40,9 @@ cudaError_t take_tc_device_error(unsigned int* flags);
 // at p = 512 or 1024, and at p = 128 from B = 64); the caller runs the in-place rdIFFT of
 // grad_c after it.
 bool circ_bwd_fused_supported(int p, int D, int64_t B);
+// Reads and clears the error word of the fused backward (bit 0: a bounded wait for its staged
+// rows timed out).
+cudaError_t take_fused_device_error(unsigned int* flags);
 cudaError_t launch_circ_bwd_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c,
                                   int64_t B, int D, int p, int dtype, cudaStream_t s);
 

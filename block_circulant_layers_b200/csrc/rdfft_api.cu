@@ -200,11 +200,12 @@ const char* rdfft_strerror(int code) {
 }
 
 int rdfft_take_device_error(void) {
-  unsigned int flags = 0, tc_flags = 0;
+  unsigned int flags = 0, tc_flags = 0, fused_flags = 0;
   cudaError_t e = rdfft::take_rows_device_error(&flags);
   if (e == cudaSuccess) e = rdfft::take_tc_device_error(&tc_flags);
+  if (e == cudaSuccess) e = rdfft::take_fused_device_error(&fused_flags);
   if (e != cudaSuccess) return finish(e);
-  return ((flags | tc_flags) & 1u) ? RDFFT_ETIMEOUT : RDFFT_OK;
+  return ((flags | tc_flags | fused_flags) & 1u) ? RDFFT_ETIMEOUT : RDFFT_OK;
 }
 
 int rdfft_selftest_wait_timeout(rdfft_stream_t stream) {

@@ -218,10 +218,12 @@ int circ_bwd_x_tc(const void* g, const float* c_hat, void* grad_x, int64_t B, in
  * No page has this; it is the library's failure detection. The row kernels move rows
  * with bulk copies and wait for them on a barrier with a bounded wait (about one
  * second): a wait that gives up leaves its rows unchanged, and records the event in a
- * word of the module's device memory instead of hanging the GPU. The tensor-core layer
- * kernels bound their waits for the tensor cores the same way (their outputs are then
- * left unwritten and their tensor memory is freed). This call reads and
- * clears that word for the current device. It synchronises with the device (a
+ * word of the module's device memory instead of hanging the GPU. The one-kernel layer
+ * backward (D = 4096 at p >= 512, 16-bit) stages its token tiles the same way (a wait that
+ * gives up leaves that CTA's remaining grad_x rows and its grad_c part unwritten, and frees
+ * its tensor memory), and the tensor-core layer kernels bound their waits for the tensor
+ * cores (their outputs are then left unwritten and their tensor memory is freed). This call
+ * reads and clears that word for the current device. It synchronises with the device (a
  * cudaMemcpyFromSymbol), so call it between steps, not inside a captured graph.
  * Returns RDFFT_OK, RDFFT_ETIMEOUT, or RDFFT_ECUDA.
  * After RDFFT_ETIMEOUT the contents of the rows of the launch that timed out are
