@@ -110,6 +110,31 @@ def test_fused_backward_p128_block_groups(rd, B, dtype):
     check_all(rd, B, 4096, 128, dtype, (150, 151 + B, 152 + B))
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B", [1, 3, 130])
+@pytest.mark.parametrize("p", [512, 1024, 2048, 4096])
+def test_fused_backward_one_block(rd, p, B, dtype):
+    """q = 1 (D = p): the one-kernel backward keeps each thread's bins of the cross-spectrum
+    in registers; ragged token tiles, one CTA storing grad_c (few tokens) or several adding."""
+    check_all(rd, B, p, p, dtype, (170 + p // 512, 171 + B, 172 + B))
+
+
+@pytest.mark.parametrize("p", [512, 4096])
+def test_fused_backward_one_block_stores_every_grad_c_element(rd, p):
+    """q = 1 with one CTA (a few tokens): grad_c is stored, not added; a NaN-filled grad_c
+    must come out finite and right."""
+    B = 3
+    c, x, g = make_layer(B, p, p, "bf16", (180, 181, 182))
+    c_hat = rd.circ_prepare(to_device(c, "f32"))
+    gc = torch.full(c_hat.shape, float("nan"), device="cuda")
+    gx = torch.empty(B, p, device="cuda", dtype=torch.bfloat16)
+    rd.circ_bwd(to_device(g, "bf16"), to_device(x, "bf16"), c_hat, p, grad_x=gx, grad_c=gc)
+    torch.cuda.synchronize()
+    gx_ref, gc_ref = oracle.circ_backward(g.exact, x.exact, c.exact)
+    assert_parity(to_host_f64(gc), gc_ref, "bf16", "one-block grad_c from NaN")
+    assert_parity(to_host_f64(gx), gx_ref, "bf16", "one-block grad_x")
+
+
 @pytest.mark.parametrize("p", [512, 1024])
 def test_fused_backward_stores_every_grad_c_element(rd, p):
     """With a single CTA (few tokens) the fused kernel stores grad_c instead of adding into a
