@@ -394,7 +394,7 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
 template <int P, typename T, int NT, int TT, int NG, int RI, int RJ>
 __global__ void __launch_bounds__(NT, 1)
 k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ grad_c,
-          int64_t B, int q, int QJ, int64_t tok_per_cta) {
+          int64_t B, int q, int QJ, int64_t tok_per_cta, int ifft_here) {
   extern __shared__ float tile[];
   constexpr int HB = P / 2;
   const int D = q * P;
@@ -487,8 +487,10 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
       if ((threadIdx.x & ~31u) % HB == 0) accumulate(true);
       else accumulate(false);
     }
-    // add this CTA's partial packed cross-spectrum into grad_c
+    // add this CTA's partial packed cross-spectrum into grad_c, or, when it owns its rows
+    // of grad_c outright, write them mirrored into the tile for the inverse below
     griddep_launch_dependents();
+    if (ifft_here) __syncthreads();                 // the last token tile is fully consumed
   #pragma unroll
     for (int n = 0; n < NG; ++n) {
       const int gam = threadIdx.x + NT * n;
@@ -504,7 +506,11 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
             float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
             const float vr = (b & 1) ? s_r[n][a][b / 2].y : s_r[n][a][b / 2].x;
             const float vi = (b & 1) ? s_i[n][a][b / 2].y : s_i[n][a][b / 2].x;
-            if (sole) {
+            if (ifft_here) {
+              const int rb = LayerGeo<P>::row_base((ib * RI + a) * QJ + jb * RJ + b);
+              tile[rb + LayerGeo<P>::at(k)] = k == 0 ? vr : vr - vi;
+              tile[rb + LayerGeo<P>::at(kim)] = k == 0 ? vi : vr + vi;
+            } else if (sole) {
               dst[k] = vr;
               dst[kim] = vi;
             } else {
@@ -575,8 +581,10 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
         }
       }
     }
-    // add this CTA's partial packed cross-spectrum into grad_c
+    // add this CTA's partial packed cross-spectrum into grad_c, or write it mirrored into
+    // the tile for the inverse below
     griddep_launch_dependents();
+    if (ifft_here) __syncthreads();                 // the last token tile is fully consumed
   #pragma unroll
     for (int n = 0; n < NG; ++n) {
       const int gam = threadIdx.x + NT * n;
@@ -590,7 +598,12 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   #pragma unroll
           for (int b = 0; b < RJ; ++b) {
             float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
-            if (sole) {
+            if (ifft_here) {
+              const int rb = LayerGeo<P>::row_base((ib * RI + a) * QJ + jb * RJ + b);
+              const float vr = s_r[n][a][b], vi = s_i[n][a][b];
+              tile[rb + LayerGeo<P>::at(k)] = k == 0 ? vr : vr - vi;
+              tile[rb + LayerGeo<P>::at(kim)] = k == 0 ? vi : vr + vi;
+            } else if (sole) {
               dst[k] = s_r[n][a][b];
               dst[kim] = s_i[n][a][b];
             } else {
@@ -600,6 +613,14 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
           }
       }
     }
+  }
+  if (ifft_here) {
+    // a CTA that covered every token owns its q x QJ rows of grad_c: their rdIFFT (Hartley
+    // form, the rows stored mirrored above) straight to grad_c, in place of a separate launch
+    __syncthreads();
+    ifft_rows_mirrored<P, NT, float>(tile, q * QJ, [&](int r) -> float* {
+      return grad_c + ((int64_t)(r / QJ) * q + j0 + r % QJ) * P;
+    });
   }
 }
 
@@ -677,7 +698,7 @@ static cudaError_t launch_x_p(const void* in, const float* chat, void* out, int6
 
 template <int P, typename T, int NT, int TT, int NG, int RI, int RJ>
 static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B, int q, int QJ,
-                          cudaStream_t s) {
+                          cudaStream_t s, bool* ifft_done) {
   auto kern = k_circ_gc<P, T, NT, TT, NG, RI, RJ>;
   const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(TT * (q + QJ));
   cudaError_t e = set_smem(kern, smem);
@@ -690,9 +711,13 @@ static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B
     e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)q * q * P, s);
     if (e != cudaSuccess) return e;
   }
+  // one token slice: each CTA owns its rows of grad_c and inverse-transforms them itself
+  // (its tile holds TT (q + QJ) rows, enough for the q QJ rows of grad_c it owns)
+  const bool here = slices == 1 && (int64_t)q * QJ <= (int64_t)TT * (q + QJ);
+  if (ifft_done) *ifft_done = here;
   dim3 grid((unsigned)slices, (unsigned)njgroups);
   return launch_pdl(kern, grid, dim3(NT), smem, s, static_cast<const T*>(g), static_cast<const T*>(x), grad_c, B,
-                    q, QJ, (int64_t)(tiles_per * TT));
+                    q, QJ, (int64_t)(tiles_per * TT), here ? 1 : 0);
 }
 
 // grad_c launcher: a CTA of 512 threads keeps S for QJ input blocks in registers,
@@ -700,52 +725,54 @@ static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B
 // at most 32 complex accumulators per thread.
 template <int P, typename T>
 static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int64_t B, int q,
-                               cudaStream_t s) {
+                               cudaStream_t s, bool* ifft_done) {
   constexpr int NT = 512;
   constexpr int TT = (P >= 2048) ? 1 : (P >= 1024 ? 2 : 4);
   constexpr int HB = P / 2;
   const int QJ = layer_qj(q, HB, 32LL * NT, (B + TT - 1) / TT, num_sms());
   if ((int64_t)HB * q * QJ > 32LL * NT) return cudaErrorInvalidConfiguration;
   const int64_t slots = (int64_t)HB * q * QJ;                // complex accumulators per CTA
-  if (q % 4 == 0 && QJ % 8 == 0 && slots <= 32LL * NT) return run_gc<P, T, NT, TT, 1, 4, 8>(g, x, grad_c, B, q, QJ, s);
+  if (q % 4 == 0 && QJ % 8 == 0 && slots <= 32LL * NT) return run_gc<P, T, NT, TT, 1, 4, 8>(g, x, grad_c, B, q, QJ, s, ifft_done);
   if (q % 4 == 0 && QJ % 4 == 0) {
-    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 1, 4, 4>(g, x, grad_c, B, q, QJ, s);
-    return run_gc<P, T, NT, TT, 2, 4, 4>(g, x, grad_c, B, q, QJ, s);
+    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 1, 4, 4>(g, x, grad_c, B, q, QJ, s, ifft_done);
+    return run_gc<P, T, NT, TT, 2, 4, 4>(g, x, grad_c, B, q, QJ, s, ifft_done);
   }
   if (q % 2 == 0 && QJ % 2 == 0) {
-    if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 1, 2, 2>(g, x, grad_c, B, q, QJ, s);
-    if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 2, 2, 2>(g, x, grad_c, B, q, QJ, s);
-    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 4, 2, 2>(g, x, grad_c, B, q, QJ, s);
-    return run_gc<P, T, NT, TT, 8, 2, 2>(g, x, grad_c, B, q, QJ, s);
+    if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 1, 2, 2>(g, x, grad_c, B, q, QJ, s, ifft_done);
+    if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 2, 2, 2>(g, x, grad_c, B, q, QJ, s, ifft_done);
+    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 4, 2, 2>(g, x, grad_c, B, q, QJ, s, ifft_done);
+    return run_gc<P, T, NT, TT, 8, 2, 2>(g, x, grad_c, B, q, QJ, s, ifft_done);
   }
-  if (slots <= 1LL * NT) return run_gc<P, T, NT, TT, 1, 1, 1>(g, x, grad_c, B, q, QJ, s);
-  if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 4, 1, 1>(g, x, grad_c, B, q, QJ, s);
-  if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 8, 1, 1>(g, x, grad_c, B, q, QJ, s);
-  if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 16, 1, 1>(g, x, grad_c, B, q, QJ, s);
-  return run_gc<P, T, NT, TT, 32, 1, 1>(g, x, grad_c, B, q, QJ, s);
+  if (slots <= 1LL * NT) return run_gc<P, T, NT, TT, 1, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
+  if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 4, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
+  if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 8, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
+  if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 16, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
+  return run_gc<P, T, NT, TT, 32, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
 }
 
 // Per-p entry of the layer, instantiated once per translation unit (circ_p*.cu):
 // op 0 = forward (a = x, out = y); op 1 = grad_x (a = g, out = grad_x);
 // op 2 = grad_c accumulation (a = g, b = x, gc = grad_c; zeroed here when several
-// token slices add into it).
+// token slices add into it). For op 2, *ifft_done (if given) tells whether the kernel also
+// ran grad_c's rdIFFT (one token slice), so the caller must not.
 template <int P>
 cudaError_t circ_layer_p(int op, const void* a, const void* b, const float* chat, void* out, float* gc,
-                         int64_t B, int q, int dtype, cudaStream_t s) {
+                         int64_t B, int q, int dtype, cudaStream_t s, bool* ifft_done) {
   if (dtype == 0) {
     if (op == 0) return launch_x_p<P, float, false>(a, chat, out, B, q, s);
     if (op == 1) return launch_x_p<P, float, true>(a, chat, out, B, q, s);
-    return launch_gc_p<P, float>(a, b, gc, B, q, s);
+    return launch_gc_p<P, float>(a, b, gc, B, q, s, ifft_done);
   }
   if (op == 0) return launch_x_p<P, bf16_t, false>(a, chat, out, B, q, s);
   if (op == 1) return launch_x_p<P, bf16_t, true>(a, chat, out, B, q, s);
-  return launch_gc_p<P, bf16_t>(a, b, gc, B, q, s);
+  return launch_gc_p<P, bf16_t>(a, b, gc, B, q, s, ifft_done);
 }
 
 #define RDFFT_CIRC_INSTANCE(PP)                                                                  \
   cudaError_t circ_layer_##PP(int op, const void* a, const void* b, const float* chat, void* out, \
-                              float* gc, int64_t B, int q, int dtype, cudaStream_t s) {           \
-    return circ_layer_p<PP>(op, a, b, chat, out, gc, B, q, dtype, s);                             \
+                              float* gc, int64_t B, int q, int dtype, cudaStream_t s,             \
+                              bool* ifft_done) {                                                  \
+    return circ_layer_p<PP>(op, a, b, chat, out, gc, B, q, dtype, s, ifft_done);                  \
   }
 
 }  // namespace rdfft
