@@ -408,106 +408,139 @@ cudaError_t run_fused(const void* g, const void* x, const float* chat, void* gra
                     static_cast<const T*>(x), chat, static_cast<T*>(grad_x), grad_c, B, (int64_t)(tiles_per * TT));
 }
 
-// The same backward for one block (q = 1, D = p): the cross-spectrum S = sum_b G conj(X) has
-// p/2 complex bins, so each thread keeps its bins' sums (and its bins' c_hat) in registers, no
-// tensor memory. A persistent CTA walks its token slice in tiles of TT tokens: rdFFT of g (tile
-// rows t) and x (rows TT + t), then per bin S += G conj(X) and the grad_x spectrum conj(C) G
-// written mirrored over the x row, then the Hartley-form rdIFFT of those rows to HBM: 3 row
-// transforms per token against 4 for the two kernels. Bin 0 holds the real pair (y_0, y_{p/2}),
-// whose products are component-wise.
-template <int P, typename T, int NT, int TT>
+// The same backward for layers of one or two blocks (q <= 2): the cross-spectrum
+// S_ij = sum_b G_i conj(X_j) has q^2 p/2 complex bins, so each thread keeps its bins' sums
+// (and its bins' c_hat) in registers, no tensor memory. A persistent CTA walks its token slice
+// in tiles of TT tokens: rdFFT of g (tile rows t q + i) and x (rows TT q + t q + j), then per bin
+// S_ij += G_i conj(X_j) and the grad_x spectra Y_j = sum_i conj(C_ij) G_i written mirrored over
+// the x rows, then the Hartley-form rdIFFT of those rows to HBM: 3 row transforms per token and
+// block against 2 + 2 for the two kernels. Bin 0 holds the real pair (y_0, y_{p/2}), whose
+// products are component-wise.
+template <int P, int Q, typename T, int NT, int TT>
 __global__ void __launch_bounds__(NT, 1)
-k_circ_bwd_q1(const T* __restrict__ g, const T* __restrict__ x, const float* __restrict__ chat,
-              T* __restrict__ grad_x, float* __restrict__ grad_c, int64_t B, int64_t tok_per_cta) {
+k_circ_bwd_small(const T* __restrict__ g, const T* __restrict__ x, const float* __restrict__ chat,
+                 T* __restrict__ grad_x, float* __restrict__ grad_c, int64_t B, int64_t tok_per_cta) {
   using G = LayerGeo<P>;
   constexpr int HB = P / 2;
   constexpr int KB = (HB + NT - 1) / NT;            // bins per thread: k = tid + NT u
-  static_assert(NT % G::TPR == 0 && (G::RW == 1 || TT % G::RW == 0), "whole rows; additive row bases");
+  constexpr int XR = TT * Q;                        // first x row of the tile
+  constexpr int D = Q * P;
+  static_assert(NT % G::TPR == 0 && (G::RW == 1 || XR % G::RW == 0), "whole rows; additive row bases");
   extern __shared__ float tile[];
   const int64_t tbeg = (int64_t)blockIdx.x * tok_per_cta;
   const int64_t tend = (tbeg + tok_per_cta < B) ? tbeg + tok_per_cta : B;
   const bool sole = (gridDim.x == 1);
   griddep_wait();
 
-  float sr[KB], si[KB], cr[KB], ci[KB];
+  float sr[KB][Q][Q], si[KB][Q][Q], cr[KB][Q][Q], ci[KB][Q][Q];
 #pragma unroll
   for (int u = 0; u < KB; ++u) {
     const int k = threadIdx.x + NT * u;
-    sr[u] = si[u] = 0.0f;
-    cr[u] = k < HB ? __ldg(chat + k) : 0.0f;
-    ci[u] = k < HB ? __ldg(chat + bin_im_slot<P>(k)) : 0.0f;
+#pragma unroll
+    for (int i = 0; i < Q; ++i)
+#pragma unroll
+      for (int j = 0; j < Q; ++j) {
+        const float* crow = chat + (int64_t)(i * Q + j) * P;
+        sr[u][i][j] = si[u][i][j] = 0.0f;
+        cr[u][i][j] = k < HB ? __ldg(crow + k) : 0.0f;
+        ci[u][i][j] = k < HB ? __ldg(crow + bin_im_slot<P>(k)) : 0.0f;
+      }
   }
   for (int64_t tok0 = tbeg; tok0 < tend; tok0 += TT) {
     const int ntok = (int)((tend - tok0) < TT ? (tend - tok0) : TT);
     if (tok0 != tbeg) __syncthreads();              // the previous tile is fully consumed
-    // 1. rdFFT of g (rows t) and x (rows TT + t)
-    fft_rows<P, NT, T>(tile, 2 * TT, [&](int r) -> const T* {
-      const int t = r < TT ? r : r - TT;
+    // 1. rdFFT of g (rows t q + i) and x (rows XR + t q + j)
+    fft_rows<P, NT, T>(tile, 2 * XR, [&](int r) -> const T* {
+      const bool isx = r >= XR;
+      const int rr = isx ? r - XR : r;
+      const int t = rr / Q, b = rr - t * Q;
       if (t >= ntok) return nullptr;
-      return (r < TT ? g : x) + (tok0 + t) * (int64_t)P;
+      return (isx ? x : g) + (tok0 + t) * (int64_t)D + (int64_t)b * P;
     });
     __syncthreads();
-    // 2. per bin: S += G conj(X); Y = conj(C) G over the x row (mirrored: slot k = Re - Im,
-    // slot p - k = Re + Im; bin 0 keeps its real pair). A thread reads and writes only its
-    // own bins' slots.
+    // 2. per bin: S_ij += G_i conj(X_j); Y_j = sum_i conj(C_ij) G_i over the x rows (mirrored:
+    // slot k = Re - Im, slot p - k = Re + Im; bin 0 keeps its real pair). A thread reads and
+    // writes only its own bins' slots.
 #pragma unroll
     for (int u = 0; u < KB; ++u) {
       const int k = threadIdx.x + NT * u;
       if (k < HB) {
         const int kr = G::at(k), ki = G::at(bin_im_slot<P>(k));
         for (int t = 0; t < ntok; ++t) {
-          const int gb = G::row_base(t), xb = G::row_base(TT + t);
-          const float gr = tile[gb + kr], gi = tile[gb + ki];
-          const float xr = tile[xb + kr], xi = tile[xb + ki];
-          if (k == 0) {
-            sr[u] = fmaf(gr, xr, sr[u]);
-            si[u] = fmaf(gi, xi, si[u]);
-            tile[xb + kr] = cr[u] * gr;
-            tile[xb + ki] = ci[u] * gi;
-          } else {
-            sr[u] = fmaf(gr, xr, fmaf(gi, xi, sr[u]));
-            si[u] = fmaf(gi, xr, fmaf(-gr, xi, si[u]));
-            const float yr = fmaf(cr[u], gr, ci[u] * gi), yi = fmaf(cr[u], gi, -(ci[u] * gr));
-            tile[xb + kr] = yr - yi;
-            tile[xb + ki] = yr + yi;
+          float gr[Q], gi[Q], xr[Q], xi[Q];
+#pragma unroll
+          for (int b = 0; b < Q; ++b) {
+            const int gb = G::row_base(t * Q + b), xb = G::row_base(XR + t * Q + b);
+            gr[b] = tile[gb + kr];
+            gi[b] = tile[gb + ki];
+            xr[b] = tile[xb + kr];
+            xi[b] = tile[xb + ki];
+          }
+#pragma unroll
+          for (int j = 0; j < Q; ++j) {
+            float yr = 0.0f, yi = 0.0f;
+#pragma unroll
+            for (int i = 0; i < Q; ++i) {
+              if (k == 0) {
+                sr[u][i][j] = fmaf(gr[i], xr[j], sr[u][i][j]);
+                si[u][i][j] = fmaf(gi[i], xi[j], si[u][i][j]);
+                yr = fmaf(cr[u][i][j], gr[i], yr);
+                yi = fmaf(ci[u][i][j], gi[i], yi);
+              } else {
+                sr[u][i][j] = fmaf(gr[i], xr[j], fmaf(gi[i], xi[j], sr[u][i][j]));
+                si[u][i][j] = fmaf(gi[i], xr[j], fmaf(-gr[i], xi[j], si[u][i][j]));
+                yr = fmaf(cr[u][i][j], gr[i], fmaf(ci[u][i][j], gi[i], yr));
+                yi = fmaf(cr[u][i][j], gi[i], fmaf(-ci[u][i][j], gr[i], yi));
+              }
+            }
+            const int xb = G::row_base(XR + t * Q + j);
+            tile[xb + kr] = k == 0 ? yr : yr - yi;
+            tile[xb + ki] = k == 0 ? yi : yr + yi;
           }
         }
       }
     }
     __syncthreads();
     // 3. rdIFFT (Hartley form) of the grad_x rows straight to HBM
-    ifft_rows_mirrored<P, NT, T>(tile + G::row_base(TT), TT, [&](int r) -> T* {
-      return r < ntok ? grad_x + (tok0 + r) * (int64_t)P : nullptr;
+    ifft_rows_mirrored<P, NT, T>(tile + G::row_base(XR), XR, [&](int r) -> T* {
+      const int t = r / Q, j = r - t * Q;
+      return t < ntok ? grad_x + (tok0 + t) * (int64_t)D + (int64_t)j * P : nullptr;
     });
   }
-  // 4. the CTA's cross-spectrum into grad_c
+  // 4. the CTA's cross-spectrum into grad_c (row i q + j)
   griddep_launch_dependents();
 #pragma unroll
   for (int u = 0; u < KB; ++u) {
     const int k = threadIdx.x + NT * u;
     if (k < HB) {
-      if (sole) {
-        grad_c[k] = sr[u];
-        grad_c[bin_im_slot<P>(k)] = si[u];
-      } else {
-        atomicAdd(grad_c + k, sr[u]);
-        atomicAdd(grad_c + bin_im_slot<P>(k), si[u]);
-      }
+#pragma unroll
+      for (int i = 0; i < Q; ++i)
+#pragma unroll
+        for (int j = 0; j < Q; ++j) {
+          float* dst = grad_c + (int64_t)(i * Q + j) * P;
+          if (sole) {
+            dst[k] = sr[u][i][j];
+            dst[bin_im_slot<P>(k)] = si[u][i][j];
+          } else {
+            atomicAdd(dst + k, sr[u][i][j]);
+            atomicAdd(dst + bin_im_slot<P>(k), si[u][i][j]);
+          }
+        }
     }
   }
 }
 
-template <int P, typename T, int NT, int TT>
-cudaError_t run_q1(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B,
-                   cudaStream_t s) {
-  auto kern = k_circ_bwd_q1<P, T, NT, TT>;
-  const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(2 * TT);
+template <int P, int Q, typename T, int NT, int TT>
+cudaError_t run_small(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B,
+                      cudaStream_t s) {
+  auto kern = k_circ_bwd_small<P, Q, T, NT, TT>;
+  const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(2 * TT * Q);
   cudaError_t e = set_smem(kern, smem);
   if (e != cudaSuccess) return e;
   int64_t tiles_per = 1;
   const int slices = layer_gc_slices(1, (B + TT - 1) / TT, num_sms(), &tiles_per);
   if (slices > 1) {
-    e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)P, s);
+    e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)Q * Q * P, s);
     if (e != cudaSuccess) return e;
   }
   return launch_pdl(kern, dim3((unsigned)slices), dim3(NT), smem, s, static_cast<const T*>(g),
@@ -518,12 +551,21 @@ template <typename T>
 cudaError_t fused_t(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B, int q,
                     int p, cudaStream_t s) {
   if (q == 1) {
-    // TT tokens per tile: 2 TT rows of TPR = p/32 threads each fill the CTA in one round
+    // TT tokens per tile: 2 TT q rows of TPR = p/32 threads each fill the CTA in one round
     switch (p) {
-      case 512: return run_q1<512, T, 128, 4>(g, x, chat, grad_x, grad_c, B, s);
-      case 1024: return run_q1<1024, T, 128, 2>(g, x, chat, grad_x, grad_c, B, s);
-      case 2048: return run_q1<2048, T, 256, 2>(g, x, chat, grad_x, grad_c, B, s);
-      case 4096: return run_q1<4096, T, 512, 2>(g, x, chat, grad_x, grad_c, B, s);
+      case 512: return run_small<512, 1, T, 128, 4>(g, x, chat, grad_x, grad_c, B, s);
+      case 1024: return run_small<1024, 1, T, 128, 2>(g, x, chat, grad_x, grad_c, B, s);
+      case 2048: return run_small<2048, 1, T, 256, 2>(g, x, chat, grad_x, grad_c, B, s);
+      case 4096: return run_small<4096, 1, T, 512, 2>(g, x, chat, grad_x, grad_c, B, s);
+      default: return cudaErrorInvalidValue;
+    }
+  }
+  if (q == 2) {
+    switch (p) {
+      case 512: return run_small<512, 2, T, 128, 2>(g, x, chat, grad_x, grad_c, B, s);
+      case 1024: return run_small<1024, 2, T, 256, 2>(g, x, chat, grad_x, grad_c, B, s);
+      case 2048: return run_small<2048, 2, T, 512, 2>(g, x, chat, grad_x, grad_c, B, s);
+      case 4096: return run_small<4096, 2, T, 512, 1>(g, x, chat, grad_x, grad_c, B, s);
       default: return cudaErrorInvalidValue;
     }
   }
@@ -546,12 +588,14 @@ cudaError_t take_fused_device_error(unsigned int* flags) {
 // p = 128 (q = 32) from 64 tokens on (backward at D = 4096: 22.9 against 26.1 us at B = 64,
 // 25.0 against 31.8 at B = 128); below, the two kernels, whose grids adapt to a handful of
 // tokens, are faster (17.9 against 19.6 us at B = 1)
-// One block (D = p) from p = 512 on, at every batch size (backward at D = p = 4096: 15.0 against
-// 17.3 us at B = 1, 15.4 against 21.7 at B = 256, 115.8 against 188.0 at B = 4096; at D = p =
-// 1024, 11.1 / 14.1 against 15.6 / 18.5 us at B = 1 / 256, even at B = 4096)
+// One or two blocks (D = p or 2 p) from p = 512 on, at every batch size (backward at D = p =
+// 4096: 15.0 against 17.3 us at B = 1, 15.4 against 21.7 at B = 256, 115.8 against 188.0 at
+// B = 4096; at D = p = 1024, 11.1 / 14.1 against 15.6 / 18.5 us at B = 1 / 256, even at B = 4096;
+// at D = 2 p = 2048, 9.2 / 12.5 / 70.3 against 13.0 / 18.8 / 121.8 us at B = 1 / 256 / 4096, and
+// at D = 2 p = 8192, 13.4 / 25.8 / 229.5 against 18.1 / 33.5 / 321.1)
 bool circ_bwd_fused_supported(int p, int D, int64_t B) {
   return (p == 512 && D == 4096) || (p == 1024 && D == 4096) || (p == 128 && D == 4096 && B >= 64) ||
-         (D == p && p >= 512);
+         ((D == p || D == 2 * p) && p >= 512);
 }
 
 cudaError_t launch_circ_bwd_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c,

@@ -119,6 +119,15 @@ def test_fused_backward_one_block(rd, p, B, dtype):
     check_all(rd, B, p, p, dtype, (170 + p // 512, 171 + B, 172 + B))
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B", [1, 3, 130])
+@pytest.mark.parametrize("p", [512, 1024, 2048, 4096])
+def test_fused_backward_two_blocks(rd, p, B, dtype):
+    """q = 2 (D = 2 p): the same register-form backward with the 2 x 2 blocks' cross-spectra
+    per bin and each grad_x block summed over both output blocks."""
+    check_all(rd, B, 2 * p, p, dtype, (190 + p // 512, 191 + B, 192 + B))
+
+
 @pytest.mark.parametrize("p", [512, 4096])
 def test_fused_backward_one_block_stores_every_grad_c_element(rd, p):
     """q = 1 with one CTA (a few tokens): grad_c is stored, not added; a NaN-filled grad_c
