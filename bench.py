@@ -410,12 +410,16 @@ def run_layer_bench(rd, torch, dev, gen, hbm_peak, fp32_peak, n_sets_bytes=256 <
                          "y": torch.empty(B, D, device=dev, dtype=dt),
                          "gx": torch.empty(B, D, device=dev, dtype=dt)})
 
+        # the deterministic backward's workspace, allocated once outside the timed graphs
+        ws = torch.empty(max(16, rd.circ_bwd_workspace_size(B, D, p, dt)), dtype=torch.uint8, device=dev)
         calls = {
             "prepare": lambda st: rd.circ_prepare(c, out=c_hat),
             "fwd": lambda st: rd.circ_fwd(st["x"], c_hat, p, y=st["y"]),
             "bwd": lambda st: rd.circ_bwd(st["g"], st["x"], c_hat, p, grad_x=st["gx"], grad_c=gc),
             "grad_x": lambda st: rd.circ_bwd(st["g"], st["x"], c_hat, p, grad_x=st["gx"], need_grad_c=False),
             "grad_c": lambda st: rd.circ_bwd(st["g"], st["x"], c_hat, p, grad_c=gc, need_grad_x=False),
+            "bwd_deterministic": lambda st: rd.circ_bwd(st["g"], st["x"], c_hat, p, grad_x=st["gx"], grad_c=gc,
+                                                        deterministic=True, workspace=ws),
         }
 
         def step_body(st):
@@ -439,7 +443,11 @@ def run_layer_bench(rd, torch, dev, gen, hbm_peak, fp32_peak, n_sets_bytes=256 <
                "bwd_tokens_s": round(B / times["bwd"], 1),
                "fwd_bwd_tokens_s": round(B / times["fwd_bwd"], 1),
                "fwd_bwd_us": round(1e6 * times["fwd_bwd"], 2),
-               "prepare_us": round(1e6 * times["prepare"], 2)}
+               "prepare_us": round(1e6 * times["prepare"], 2),
+               # circ_bwd_deterministic: grad_c's token slices summed in order via a workspace
+               "bwd_deterministic": {"us": round(1e6 * times["bwd_deterministic"], 2),
+                                     "workspace_MiB": round(ws.numel() / 2**20, 2),
+                                     "vs_bwd": round(times["bwd"] / times["bwd_deterministic"], 3)}}
         for key in ("fwd", "bwd", "grad_x", "grad_c"):
             t = times[key]
             w = work[key]

@@ -13,7 +13,8 @@ Tensor functions (torch is used for device memory and the current stream):
     rdfft_from_complex(z)                 packed rows from complex bins, out of place
     rdfft2_fwd(t) / rdfft2_inv(t)         in place, 2-D packed spectrum of (..., R, C)
     circ_fwd(x, c_hat, p, y=None)         y = W x
-    circ_bwd(g, x, c_hat, p, grad_x=..., grad_c=...)
+    circ_bwd(g, x, c_hat, p, grad_x=..., grad_c=..., deterministic=False)
+    circ_bwd_workspace_size(B, D, p, dtype)  device bytes the deterministic backward needs
     circ_prepare(c)                       c_hat = packed rdfft_fwd of fp32 c
     circ_fwd_tc / circ_bwd_x_tc           forward / grad_x with the contraction on the tensor
                                           cores (bf16, p = 128, D = 4096; slower, kept measured)
@@ -23,7 +24,7 @@ Raw entry points on integer device pointers: ``lib`` (the ctypes handle).
 from __future__ import annotations
 
 _EXPORTS = ("RDFFT_BF16", "RDFFT_F32", "RDFFT_ETIMEOUT", "RdfftError", "circ_bwd", "circ_fwd", "circ_prepare",
-            "circ_fwd_tc", "circ_bwd_x_tc",
+            "circ_fwd_tc", "circ_bwd_x_tc", "circ_bwd_workspace_size",
             "lib", "lib_path", "rdfft_fwd", "rdfft_inv", "rdfft_to_complex", "rdfft_from_complex", "rdfft2_fwd",
             "rdfft2_inv", "take_device_error", "selftest_wait_timeout")
 _LAYER = ("BlockCirculantLinear", "block_circulant")

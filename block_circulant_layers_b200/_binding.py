@@ -31,8 +31,11 @@ lib.circ_fwd.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_bwd.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_fwd_tc.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_bwd_x_tc.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
+lib.circ_bwd_workspace_size.argtypes = [_i64, _int, _int, _int, _int, ctypes.POINTER(ctypes.c_size_t)]
+lib.circ_bwd_deterministic.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _vp, ctypes.c_size_t, _vp]
 for _f in (lib.rdfft_fwd, lib.rdfft_inv, lib.rdfft_to_complex, lib.rdfft_from_complex, lib.rdfft2_fwd,
-           lib.rdfft2_inv, lib.circ_prepare, lib.circ_fwd, lib.circ_bwd, lib.circ_fwd_tc, lib.circ_bwd_x_tc):
+           lib.rdfft2_inv, lib.circ_prepare, lib.circ_fwd, lib.circ_bwd, lib.circ_fwd_tc, lib.circ_bwd_x_tc,
+           lib.circ_bwd_workspace_size, lib.circ_bwd_deterministic):
     _f.restype = _int
 lib.rdfft_strerror.argtypes = [_int]
 lib.rdfft_strerror.restype = ctypes.c_char_p
@@ -202,10 +205,23 @@ def circ_fwd(x: torch.Tensor, c_hat: torch.Tensor, p: int, y: torch.Tensor | Non
     return y
 
 
+def circ_bwd_workspace_size(B: int, D: int, p: int, dtype: torch.dtype, with_grad_x: bool = True) -> int:
+    """Bytes of workspace circ_bwd(..., deterministic=True) needs on the current device (0: none)."""
+    n = ctypes.c_size_t()
+    code = RDFFT_BF16 if dtype == torch.bfloat16 else RDFFT_F32
+    _check(lib.circ_bwd_workspace_size(B, D, p, code, int(with_grad_x), ctypes.byref(n)), "circ_bwd_workspace_size")
+    return n.value
+
+
 def circ_bwd(g: torch.Tensor, x: torch.Tensor, c_hat: torch.Tensor, p: int,
              grad_x: torch.Tensor | None = None, grad_c: torch.Tensor | None = None,
-             need_grad_x: bool = True, need_grad_c: bool = True):
-    """(grad_x, grad_c) of the block-circulant layer for upstream gradient g."""
+             need_grad_x: bool = True, need_grad_c: bool = True, deterministic: bool = False,
+             workspace: torch.Tensor | None = None):
+    """(grad_x, grad_c) of the block-circulant layer for upstream gradient g.
+
+    deterministic=True calls circ_bwd_deterministic: grad_c is then the same bit for bit
+    from run to run. Its workspace (device bytes, circ_bwd_workspace_size) is taken from
+    `workspace` if given, else allocated here through torch's caching allocator."""
     _cuda_dense(g, "g")
     _cuda_dense(x, "x")
     _cuda_dense(c_hat, "c_hat")
@@ -221,8 +237,18 @@ def circ_bwd(g: torch.Tensor, x: torch.Tensor, c_hat: torch.Tensor, p: int,
     gx_ptr = grad_x.data_ptr() if (need_grad_x and grad_x is not None) else None
     gc_ptr = grad_c.data_ptr() if (need_grad_c and grad_c is not None) else None
     with torch.cuda.device(x.device):
-        _check(lib.circ_bwd(g.data_ptr(), x.data_ptr(), c_hat.data_ptr(), gx_ptr, gc_ptr, B, D, p,
-                            _dtype_code(x), _stream(x)), "circ_bwd")
+        if not deterministic:
+            _check(lib.circ_bwd(g.data_ptr(), x.data_ptr(), c_hat.data_ptr(), gx_ptr, gc_ptr, B, D, p,
+                                _dtype_code(x), _stream(x)), "circ_bwd")
+        else:
+            need = circ_bwd_workspace_size(B, D, p, x.dtype, gx_ptr is not None) if gc_ptr is not None else 0
+            if workspace is None:
+                workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=x.device)
+            _cuda_dense(workspace, "workspace")
+            _check(lib.circ_bwd_deterministic(g.data_ptr(), x.data_ptr(), c_hat.data_ptr(), gx_ptr, gc_ptr, B, D,
+                                              p, _dtype_code(x), workspace.data_ptr(),
+                                              workspace.numel() * workspace.element_size(), _stream(x)),
+                   "circ_bwd_deterministic")
     return (grad_x if need_grad_x else None), (grad_c if need_grad_c else None)
 
 

@@ -58,7 +58,8 @@ struct FusedSmem {
 template <int P, int Q, int QJ, typename T, int NT, int TT, int RI, int RJ>
 __global__ void __launch_bounds__(NT, 1)
 k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* __restrict__ chat,
-                 T* __restrict__ grad_x, float* __restrict__ grad_c, int64_t B, int64_t tok_per_cta) {
+                 T* __restrict__ grad_x, float* __restrict__ grad_c, float* __restrict__ partial, int64_t B,
+                 int64_t tok_per_cta) {
   using G = LayerGeo<P>;
   constexpr int q = Q;
   constexpr int HB = P / 2;
@@ -81,7 +82,10 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
   const int D = q * P;
   const int64_t tbeg = (int64_t)blockIdx.x * tok_per_cta;
   const int64_t tend = (tbeg + tok_per_cta < B) ? tbeg + tok_per_cta : B;
-  const bool sole = (gridDim.x == 1);
+  // one token slice stores its sums (they are final); with per-slice sums (partial) every
+  // slice stores its own q x q x p spectrum the same way; otherwise the slices add
+  const bool store = (gridDim.x == 1) || partial != nullptr;
+  float* const gc_base = partial != nullptr ? partial + (int64_t)blockIdx.x * q * q * P : grad_c;
   const int warp = threadIdx.x >> 5;
   const int j0 = blockIdx.y * QJ;                   // the group's first input block
   const int nib = q / RI;
@@ -371,10 +375,10 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
     for (int a = 0; a < RI; ++a)
 #pragma unroll
       for (int b = 0; b < RJ; ++b) {
-        float* dst = grad_c + ((int64_t)(gib * RI + a) * q + (j0 + gjb * RJ + b)) * P;
+        float* dst = gc_base + ((int64_t)(gib * RI + a) * q + (j0 + gjb * RJ + b)) * P;
         const int o = (a * RJP + b / 2) * 4 + (b & 1);
         const float vr = acc[o], vi = acc[o + 2];
-        if (sole) {
+        if (store) {
           dst[gk] = vr;
           dst[kim] = vi;
         } else {
@@ -390,22 +394,26 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
 
 template <int P, int Q, int QJ, typename T, int TT, int RI, int RJ>
 cudaError_t run_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B,
-                      cudaStream_t s) {
+                      cudaStream_t s, GcSink* sink) {
   constexpr int NT = 512;
   constexpr int q = Q;
   auto kern = k_circ_bwd_fused<P, Q, QJ, T, NT, TT, RI, RJ>;
   const size_t smem = FusedSmem<P, Q, QJ, T, TT>::BYTES;
-  cudaError_t e = set_smem(kern, smem);
-  if (e != cudaSuccess) return e;
   constexpr int NJG = Q / QJ;                      // input-block groups
   int64_t tiles_per = 1;
   const int slices = layer_gc_slices(NJG, (B + TT - 1) / TT, num_sms(), &tiles_per);
-  if (slices > 1) {
-    e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)q * q * P, s);
+  float* partial = nullptr;
+  cudaError_t e = sink_plan(sink, slices, (int64_t)q * q * P, &partial);
+  if (e != cudaSuccess || (sink && sink->plan_only)) return e;
+  e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  if (slices > 1 && !partial) {
+    e = launch_zero_f32(grad_c, (int64_t)q * q * P, s);
     if (e != cudaSuccess) return e;
   }
   return launch_pdl(kern, dim3((unsigned)slices, (unsigned)NJG), dim3(NT), smem, s, static_cast<const T*>(g),
-                    static_cast<const T*>(x), chat, static_cast<T*>(grad_x), grad_c, B, (int64_t)(tiles_per * TT));
+                    static_cast<const T*>(x), chat, static_cast<T*>(grad_x), grad_c, partial, B,
+                    (int64_t)(tiles_per * TT));
 }
 
 // The same backward for layers of one or two blocks (q <= 2): the cross-spectrum
@@ -419,7 +427,8 @@ cudaError_t run_fused(const void* g, const void* x, const float* chat, void* gra
 template <int P, int Q, typename T, int NT, int TT>
 __global__ void __launch_bounds__(NT, 1)
 k_circ_bwd_small(const T* __restrict__ g, const T* __restrict__ x, const float* __restrict__ chat,
-                 T* __restrict__ grad_x, float* __restrict__ grad_c, int64_t B, int64_t tok_per_cta) {
+                 T* __restrict__ grad_x, float* __restrict__ grad_c, float* __restrict__ partial, int64_t B,
+                 int64_t tok_per_cta) {
   using G = LayerGeo<P>;
   constexpr int HB = P / 2;
   constexpr int KB = (HB + NT - 1) / NT;            // bins per thread: k = tid + NT u
@@ -429,7 +438,8 @@ k_circ_bwd_small(const T* __restrict__ g, const T* __restrict__ x, const float* 
   extern __shared__ float tile[];
   const int64_t tbeg = (int64_t)blockIdx.x * tok_per_cta;
   const int64_t tend = (tbeg + tok_per_cta < B) ? tbeg + tok_per_cta : B;
-  const bool sole = (gridDim.x == 1);
+  const bool store = (gridDim.x == 1) || partial != nullptr;   // as in k_circ_bwd_fused
+  float* const gc_base = partial != nullptr ? partial + (int64_t)blockIdx.x * Q * Q * P : grad_c;
   griddep_wait();
 
   float sr[KB][Q][Q], si[KB][Q][Q], cr[KB][Q][Q], ci[KB][Q][Q];
@@ -517,8 +527,8 @@ k_circ_bwd_small(const T* __restrict__ g, const T* __restrict__ x, const float* 
       for (int i = 0; i < Q; ++i)
 #pragma unroll
         for (int j = 0; j < Q; ++j) {
-          float* dst = grad_c + (int64_t)(i * Q + j) * P;
-          if (sole) {
+          float* dst = gc_base + (int64_t)(i * Q + j) * P;
+          if (store) {
             dst[k] = sr[u][i][j];
             dst[bin_im_slot<P>(k)] = si[u][i][j];
           } else {
@@ -532,46 +542,50 @@ k_circ_bwd_small(const T* __restrict__ g, const T* __restrict__ x, const float* 
 
 template <int P, int Q, typename T, int NT, int TT>
 cudaError_t run_small(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B,
-                      cudaStream_t s) {
+                      cudaStream_t s, GcSink* sink) {
   auto kern = k_circ_bwd_small<P, Q, T, NT, TT>;
   const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(2 * TT * Q);
-  cudaError_t e = set_smem(kern, smem);
-  if (e != cudaSuccess) return e;
   int64_t tiles_per = 1;
   const int slices = layer_gc_slices(1, (B + TT - 1) / TT, num_sms(), &tiles_per);
-  if (slices > 1) {
-    e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)Q * Q * P, s);
+  float* partial = nullptr;
+  cudaError_t e = sink_plan(sink, slices, (int64_t)Q * Q * P, &partial);
+  if (e != cudaSuccess || (sink && sink->plan_only)) return e;
+  e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  if (slices > 1 && !partial) {
+    e = launch_zero_f32(grad_c, (int64_t)Q * Q * P, s);
     if (e != cudaSuccess) return e;
   }
   return launch_pdl(kern, dim3((unsigned)slices), dim3(NT), smem, s, static_cast<const T*>(g),
-                    static_cast<const T*>(x), chat, static_cast<T*>(grad_x), grad_c, B, (int64_t)(tiles_per * TT));
+                    static_cast<const T*>(x), chat, static_cast<T*>(grad_x), grad_c, partial, B,
+                    (int64_t)(tiles_per * TT));
 }
 
 template <typename T>
 cudaError_t fused_t(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c, int64_t B, int q,
-                    int p, cudaStream_t s) {
+                    int p, cudaStream_t s, GcSink* sink) {
   if (q == 1) {
     // TT tokens per tile: 2 TT q rows of TPR = p/32 threads each fill the CTA in one round
     switch (p) {
-      case 512: return run_small<512, 1, T, 128, 4>(g, x, chat, grad_x, grad_c, B, s);
-      case 1024: return run_small<1024, 1, T, 128, 2>(g, x, chat, grad_x, grad_c, B, s);
-      case 2048: return run_small<2048, 1, T, 256, 2>(g, x, chat, grad_x, grad_c, B, s);
-      case 4096: return run_small<4096, 1, T, 512, 2>(g, x, chat, grad_x, grad_c, B, s);
+      case 512: return run_small<512, 1, T, 128, 4>(g, x, chat, grad_x, grad_c, B, s, sink);
+      case 1024: return run_small<1024, 1, T, 128, 2>(g, x, chat, grad_x, grad_c, B, s, sink);
+      case 2048: return run_small<2048, 1, T, 256, 2>(g, x, chat, grad_x, grad_c, B, s, sink);
+      case 4096: return run_small<4096, 1, T, 512, 2>(g, x, chat, grad_x, grad_c, B, s, sink);
       default: return cudaErrorInvalidValue;
     }
   }
   if (q == 2) {
     switch (p) {
-      case 512: return run_small<512, 2, T, 128, 2>(g, x, chat, grad_x, grad_c, B, s);
-      case 1024: return run_small<1024, 2, T, 256, 2>(g, x, chat, grad_x, grad_c, B, s);
-      case 2048: return run_small<2048, 2, T, 512, 2>(g, x, chat, grad_x, grad_c, B, s);
-      case 4096: return run_small<4096, 2, T, 512, 1>(g, x, chat, grad_x, grad_c, B, s);
+      case 512: return run_small<512, 2, T, 128, 2>(g, x, chat, grad_x, grad_c, B, s, sink);
+      case 1024: return run_small<1024, 2, T, 256, 2>(g, x, chat, grad_x, grad_c, B, s, sink);
+      case 2048: return run_small<2048, 2, T, 512, 2>(g, x, chat, grad_x, grad_c, B, s, sink);
+      case 4096: return run_small<4096, 2, T, 512, 1>(g, x, chat, grad_x, grad_c, B, s, sink);
       default: return cudaErrorInvalidValue;
     }
   }
-  if (p == 128 && q == 32) return run_fused<128, 32, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s);
-  if (p == 512 && q == 8) return run_fused<512, 8, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s);
-  if (p == 1024 && q == 4) return run_fused<1024, 4, 4, T, 2, 4, 4>(g, x, chat, grad_x, grad_c, B, s);
+  if (p == 128 && q == 32) return run_fused<128, 32, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s, sink);
+  if (p == 512 && q == 8) return run_fused<512, 8, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s, sink);
+  if (p == 1024 && q == 4) return run_fused<1024, 4, 4, T, 2, 4, 4>(g, x, chat, grad_x, grad_c, B, s, sink);
   return cudaErrorInvalidValue;
 }
 
@@ -599,10 +613,10 @@ bool circ_bwd_fused_supported(int p, int D, int64_t B) {
 }
 
 cudaError_t launch_circ_bwd_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c,
-                                  int64_t B, int D, int p, int dtype, cudaStream_t s) {
+                                  int64_t B, int D, int p, int dtype, cudaStream_t s, GcSink* sink) {
   const int q = D / p;
-  if (dtype == 0) return fused_t<float>(g, x, chat, grad_x, grad_c, B, q, p, s);
-  return fused_t<bf16_t>(g, x, chat, grad_x, grad_c, B, q, p, s);
+  if (dtype == 0) return fused_t<float>(g, x, chat, grad_x, grad_c, B, q, p, s, sink);
+  return fused_t<bf16_t>(g, x, chat, grad_x, grad_c, B, q, p, s, sink);
 }
 
 }  // namespace rdfft

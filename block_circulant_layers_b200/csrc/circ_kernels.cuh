@@ -394,7 +394,7 @@ k_circ_x(const T* __restrict__ in, const float* __restrict__ chat, T* __restrict
 template <int P, typename T, int NT, int TT, int NG, int RI, int RJ>
 __global__ void __launch_bounds__(NT, 1)
 k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ grad_c,
-          int64_t B, int q, int QJ, int64_t tok_per_cta, int ifft_here) {
+          float* __restrict__ partial, int64_t B, int q, int QJ, int64_t tok_per_cta, int ifft_here) {
   extern __shared__ float tile[];
   constexpr int HB = P / 2;
   const int D = q * P;
@@ -404,8 +404,10 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
   const int nib = q / RI, njb = QJ / RJ;
   const int ngroups = HB * nib * njb;
   // the only token slice: this CTA's sums are final and every (bin, i, j) of its group
-  // is one thread-group's, so it stores them instead of adding into a zeroed grad_c
-  const bool sole = (gridDim.x == 1);
+  // is one thread-group's, so it stores them instead of adding into a zeroed grad_c; with
+  // per-slice sums (partial), each slice stores its own q x q x p spectrum the same way
+  const bool store = (gridDim.x == 1) || partial != nullptr;
+  float* const gc_base = partial != nullptr ? partial + (int64_t)blockIdx.x * q * q * P : grad_c;
   griddep_wait();                            // earlier work in the stream (g, x, zeroed grad_c) is done
 
   if constexpr (RJ % 2 == 0) {
@@ -503,14 +505,14 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
         for (int a = 0; a < RI; ++a)
   #pragma unroll
           for (int b = 0; b < RJ; ++b) {
-            float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
+            float* dst = gc_base + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
             const float vr = (b & 1) ? s_r[n][a][b / 2].y : s_r[n][a][b / 2].x;
             const float vi = (b & 1) ? s_i[n][a][b / 2].y : s_i[n][a][b / 2].x;
             if (ifft_here) {
               const int rb = LayerGeo<P>::row_base((ib * RI + a) * QJ + jb * RJ + b);
               tile[rb + LayerGeo<P>::at(k)] = k == 0 ? vr : vr - vi;
               tile[rb + LayerGeo<P>::at(kim)] = k == 0 ? vi : vr + vi;
-            } else if (sole) {
+            } else if (store) {
               dst[k] = vr;
               dst[kim] = vi;
             } else {
@@ -597,13 +599,13 @@ k_circ_gc(const T* __restrict__ g, const T* __restrict__ x, float* __restrict__ 
         for (int a = 0; a < RI; ++a)
   #pragma unroll
           for (int b = 0; b < RJ; ++b) {
-            float* dst = grad_c + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
+            float* dst = gc_base + ((int64_t)(ib * RI + a) * q + (j0 + jb * RJ + b)) * P;
             if (ifft_here) {
               const int rb = LayerGeo<P>::row_base((ib * RI + a) * QJ + jb * RJ + b);
               const float vr = s_r[n][a][b], vi = s_i[n][a][b];
               tile[rb + LayerGeo<P>::at(k)] = k == 0 ? vr : vr - vi;
               tile[rb + LayerGeo<P>::at(kim)] = k == 0 ? vi : vr + vi;
-            } else if (sole) {
+            } else if (store) {
               dst[k] = s_r[n][a][b];
               dst[kim] = s_i[n][a][b];
             } else {
@@ -696,28 +698,62 @@ static cudaError_t launch_x_p(const void* in, const float* chat, void* out, int6
   }
 }
 
+// grad_c := 0 before several token slices add into it. A kernel rather than a memset, so the
+// launch chains with programmatic dependent launch like the kernels around it (in a CUDA
+// graph a memset node does not). n is q^2 p, a multiple of 64; p is 16-byte aligned.
+static __global__ void __launch_bounds__(256) k_zero_f4(float4* __restrict__ p, int64_t n4) {
+  griddep_wait();                                  // earlier readers of the buffer are done
+  for (int64_t i = (int64_t)blockIdx.x * 256 + threadIdx.x; i < n4; i += (int64_t)gridDim.x * 256)
+    p[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+  griddep_launch_dependents();
+}
+
+static cudaError_t launch_zero_f32(float* p, int64_t n, cudaStream_t s) {
+  const int64_t n4 = n / 4;
+  int64_t blocks = (n4 + 255) / 256;
+  if (blocks > 4 * 148) blocks = 4 * 148;
+  return launch_pdl(k_zero_f4, dim3((unsigned)blocks), dim3(256), 0, s, reinterpret_cast<float4*>(p), n4);
+}
+
+// Records the launch shape in the sink and picks where the slices' sums go: the sink's
+// partial buffer when there are several slices and one was given (its capacity checked),
+// else nothing (the kernel stores into grad_c with one slice, or adds into it).
+static cudaError_t sink_plan(GcSink* sink, int slices, int64_t floats_per_slice, float** partial) {
+  *partial = nullptr;
+  if (sink == nullptr) return cudaSuccess;
+  sink->slices = slices;
+  sink->ifft_done = false;
+  if (sink->plan_only || slices <= 1 || sink->partial == nullptr) return cudaSuccess;
+  if ((int64_t)slices * floats_per_slice > sink->partial_floats) return cudaErrorInvalidValue;
+  *partial = sink->partial;
+  return cudaSuccess;
+}
+
 template <int P, typename T, int NT, int TT, int NG, int RI, int RJ>
 static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B, int q, int QJ,
-                          cudaStream_t s, bool* ifft_done) {
+                          cudaStream_t s, GcSink* sink) {
   auto kern = k_circ_gc<P, T, NT, TT, NG, RI, RJ>;
   const size_t smem = sizeof(float) * (size_t)LayerGeo<P>::words(TT * (q + QJ));
-  cudaError_t e = set_smem(kern, smem);
-  if (e != cudaSuccess) return e;
   const int njgroups = q / QJ;
   int64_t tiles_per = 1;
   const int slices = layer_gc_slices(njgroups, (B + TT - 1) / TT, num_sms(), &tiles_per);
-  if (slices > 1) {
-    // several token slices add their partial sums into grad_c; one slice stores them
-    e = cudaMemsetAsync(grad_c, 0, sizeof(float) * (size_t)q * q * P, s);
-    if (e != cudaSuccess) return e;
-  }
   // one token slice: each CTA owns its rows of grad_c and inverse-transforms them itself
   // (its tile holds TT (q + QJ) rows, enough for the q QJ rows of grad_c it owns)
   const bool here = slices == 1 && (int64_t)q * QJ <= (int64_t)TT * (q + QJ);
-  if (ifft_done) *ifft_done = here;
+  float* partial = nullptr;
+  cudaError_t e = sink_plan(sink, slices, (int64_t)q * q * P, &partial);
+  if (sink) sink->ifft_done = here;
+  if (e != cudaSuccess || (sink && sink->plan_only)) return e;
+  e = set_smem(kern, smem);
+  if (e != cudaSuccess) return e;
+  if (slices > 1 && !partial) {
+    // several token slices add their partial sums into grad_c; one slice stores them
+    e = launch_zero_f32(grad_c, (int64_t)q * q * P, s);
+    if (e != cudaSuccess) return e;
+  }
   dim3 grid((unsigned)slices, (unsigned)njgroups);
-  return launch_pdl(kern, grid, dim3(NT), smem, s, static_cast<const T*>(g), static_cast<const T*>(x), grad_c, B,
-                    q, QJ, (int64_t)(tiles_per * TT), here ? 1 : 0);
+  return launch_pdl(kern, grid, dim3(NT), smem, s, static_cast<const T*>(g), static_cast<const T*>(x), grad_c,
+                    partial, B, q, QJ, (int64_t)(tiles_per * TT), here ? 1 : 0);
 }
 
 // grad_c launcher: a CTA of 512 threads keeps S for QJ input blocks in registers,
@@ -725,54 +761,55 @@ static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B
 // at most 32 complex accumulators per thread.
 template <int P, typename T>
 static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int64_t B, int q,
-                               cudaStream_t s, bool* ifft_done) {
+                               cudaStream_t s, GcSink* sink) {
   constexpr int NT = 512;
   constexpr int TT = (P >= 2048) ? 1 : (P >= 1024 ? 2 : 4);
   constexpr int HB = P / 2;
   const int QJ = layer_qj(q, HB, 32LL * NT, (B + TT - 1) / TT, num_sms());
   if ((int64_t)HB * q * QJ > 32LL * NT) return cudaErrorInvalidConfiguration;
   const int64_t slots = (int64_t)HB * q * QJ;                // complex accumulators per CTA
-  if (q % 4 == 0 && QJ % 8 == 0 && slots <= 32LL * NT) return run_gc<P, T, NT, TT, 1, 4, 8>(g, x, grad_c, B, q, QJ, s, ifft_done);
+  if (q % 4 == 0 && QJ % 8 == 0 && slots <= 32LL * NT) return run_gc<P, T, NT, TT, 1, 4, 8>(g, x, grad_c, B, q, QJ, s, sink);
   if (q % 4 == 0 && QJ % 4 == 0) {
-    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 1, 4, 4>(g, x, grad_c, B, q, QJ, s, ifft_done);
-    return run_gc<P, T, NT, TT, 2, 4, 4>(g, x, grad_c, B, q, QJ, s, ifft_done);
+    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 1, 4, 4>(g, x, grad_c, B, q, QJ, s, sink);
+    return run_gc<P, T, NT, TT, 2, 4, 4>(g, x, grad_c, B, q, QJ, s, sink);
   }
   if (q % 2 == 0 && QJ % 2 == 0) {
-    if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 1, 2, 2>(g, x, grad_c, B, q, QJ, s, ifft_done);
-    if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 2, 2, 2>(g, x, grad_c, B, q, QJ, s, ifft_done);
-    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 4, 2, 2>(g, x, grad_c, B, q, QJ, s, ifft_done);
-    return run_gc<P, T, NT, TT, 8, 2, 2>(g, x, grad_c, B, q, QJ, s, ifft_done);
+    if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 1, 2, 2>(g, x, grad_c, B, q, QJ, s, sink);
+    if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 2, 2, 2>(g, x, grad_c, B, q, QJ, s, sink);
+    if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 4, 2, 2>(g, x, grad_c, B, q, QJ, s, sink);
+    return run_gc<P, T, NT, TT, 8, 2, 2>(g, x, grad_c, B, q, QJ, s, sink);
   }
-  if (slots <= 1LL * NT) return run_gc<P, T, NT, TT, 1, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
-  if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 4, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
-  if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 8, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
-  if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 16, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
-  return run_gc<P, T, NT, TT, 32, 1, 1>(g, x, grad_c, B, q, QJ, s, ifft_done);
+  if (slots <= 1LL * NT) return run_gc<P, T, NT, TT, 1, 1, 1>(g, x, grad_c, B, q, QJ, s, sink);
+  if (slots <= 4LL * NT) return run_gc<P, T, NT, TT, 4, 1, 1>(g, x, grad_c, B, q, QJ, s, sink);
+  if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 8, 1, 1>(g, x, grad_c, B, q, QJ, s, sink);
+  if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 16, 1, 1>(g, x, grad_c, B, q, QJ, s, sink);
+  return run_gc<P, T, NT, TT, 32, 1, 1>(g, x, grad_c, B, q, QJ, s, sink);
 }
 
 // Per-p entry of the layer, instantiated once per translation unit (circ_p*.cu):
 // op 0 = forward (a = x, out = y); op 1 = grad_x (a = g, out = grad_x);
 // op 2 = grad_c accumulation (a = g, b = x, gc = grad_c; zeroed here when several
-// token slices add into it). For op 2, *ifft_done (if given) tells whether the kernel also
-// ran grad_c's rdIFFT (one token slice), so the caller must not.
+// token slices add into it). For op 2, the sink (if given) receives the slice count and
+// whether the kernel also ran grad_c's rdIFFT (one token slice), so the caller must not; its
+// partial buffer, if set, takes the slices' sums instead of atomics into grad_c.
 template <int P>
 cudaError_t circ_layer_p(int op, const void* a, const void* b, const float* chat, void* out, float* gc,
-                         int64_t B, int q, int dtype, cudaStream_t s, bool* ifft_done) {
+                         int64_t B, int q, int dtype, cudaStream_t s, GcSink* sink) {
   if (dtype == 0) {
     if (op == 0) return launch_x_p<P, float, false>(a, chat, out, B, q, s);
     if (op == 1) return launch_x_p<P, float, true>(a, chat, out, B, q, s);
-    return launch_gc_p<P, float>(a, b, gc, B, q, s, ifft_done);
+    return launch_gc_p<P, float>(a, b, gc, B, q, s, sink);
   }
   if (op == 0) return launch_x_p<P, bf16_t, false>(a, chat, out, B, q, s);
   if (op == 1) return launch_x_p<P, bf16_t, true>(a, chat, out, B, q, s);
-  return launch_gc_p<P, bf16_t>(a, b, gc, B, q, s, ifft_done);
+  return launch_gc_p<P, bf16_t>(a, b, gc, B, q, s, sink);
 }
 
 #define RDFFT_CIRC_INSTANCE(PP)                                                                  \
   cudaError_t circ_layer_##PP(int op, const void* a, const void* b, const float* chat, void* out, \
                               float* gc, int64_t B, int q, int dtype, cudaStream_t s,             \
-                              bool* ifft_done) {                                                  \
-    return circ_layer_p<PP>(op, a, b, chat, out, gc, B, q, dtype, s, ifft_done);                  \
+                              GcSink* sink) {                                                     \
+    return circ_layer_p<PP>(op, a, b, chat, out, gc, B, q, dtype, s, sink);                       \
   }
 
 }  // namespace rdfft

@@ -35,23 +35,42 @@ bool circ_tc_supported(int p, int D, int dtype);
 cudaError_t launch_circ_x_tc(const void* in, const float* chat, void* out, int64_t B, bool bwdx, cudaStream_t s);
 cudaError_t take_tc_device_error(unsigned int* flags);
 
+// Where a grad_c launch puts its token slices' sums, and what it reports back. Without a
+// sink (or with partial == nullptr) several slices add into a zeroed grad_c with fp32
+// atomics; with partial, slice s stores its packed sums at partial + s q^2 p (the whole
+// q x q x p spectrum over the slice's block groups) and the caller sums the slices in order.
+struct GcSink {
+  float* partial = nullptr;      // in: per-slice sums (deterministic mode), or nullptr
+  int64_t partial_floats = 0;    // in: capacity of partial
+  bool plan_only = false;        // in: work out the launch shape, enqueue nothing
+  int slices = 0;                // out: token slices of the grad_c launch
+  bool ifft_done = false;        // out: the kernel also ran grad_c's rdIFFT (one slice)
+};
+
 // Backward in one kernel (grad_x and the grad_c cross-spectrum from one transform of g
 // and x per input-block group) for the shapes it covers (circ_bwd_fused_supported: D = 4096
-// at p = 512 or 1024, at p = 128 from B = 64, and one-block layers D = p >= 512); the caller
-// runs the in-place rdIFFT of grad_c after it.
+// at p = 512 or 1024, at p = 128 from B = 64, and layers of one or two blocks, D in {p, 2p},
+// p >= 512); the caller runs the in-place rdIFFT of grad_c after it.
 bool circ_bwd_fused_supported(int p, int D, int64_t B);
 // Reads and clears the error word of the fused backward (bit 0: a bounded wait for its staged
 // rows timed out).
 cudaError_t take_fused_device_error(unsigned int* flags);
 cudaError_t launch_circ_bwd_fused(const void* g, const void* x, const float* chat, void* grad_x, float* grad_c,
-                                  int64_t B, int D, int p, int dtype, cudaStream_t s);
+                                  int64_t B, int D, int p, int dtype, cudaStream_t s, GcSink* sink);
 
 // Block-circulant layer forward: y = W x (see circ_fwd in rdfft.h).
 cudaError_t launch_circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p,
                             int dtype, cudaStream_t s);
 
 // Block-circulant layer backward (see circ_bwd in rdfft.h). grad_x / grad_c may be null.
+// With a sink whose partial is set, grad_c's token slices are summed in slice order (see
+// circ_bwd_deterministic).
 cudaError_t launch_circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x,
-                            float* grad_c, int64_t B, int D, int p, int dtype, cudaStream_t s);
+                            float* grad_c, int64_t B, int D, int p, int dtype, cudaStream_t s,
+                            GcSink* sink = nullptr);
+
+// Token slices of the grad_c launch that launch_circ_bwd would make for these sizes with
+// grad_c requested (and grad_x too if with_grad_x); enqueues nothing.
+cudaError_t plan_circ_bwd(int64_t B, int D, int p, int dtype, bool with_grad_x, int* slices);
 
 }  // namespace rdfft

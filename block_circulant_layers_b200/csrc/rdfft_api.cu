@@ -79,6 +79,38 @@ int image_call(void* data, int64_t images, int R, int C, int dtype, rdfft_stream
   return finish(rdfft::launch_rows(data, rows, C, dtype, true, s));
 }
 
+// Bytes of c_hat or grad_c: q x q x p fp32.
+size_t gc_bytes(int D, int p) { return sizeof(float) * (size_t)(D / p) * (D / p) * p; }
+
+// Argument checks of the layer backward (circ_bwd, circ_bwd_deterministic). Returns
+// kEnqueue when the call has work to enqueue, else the call's return code (an error, or
+// RDFFT_OK when there is nothing to do or an empty batch only zeroed grad_c).
+constexpr int kEnqueue = -1;
+int bwd_args(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c, int64_t B, int D,
+             int p, int dtype, rdfft_stream_t stream) {
+  if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
+  if (!layer_shape_ok(B, D, p)) return RDFFT_EINVAL;
+  if (grad_x == nullptr && grad_c == nullptr) return RDFFT_OK;
+  const size_t cb = gc_bytes(D, p);
+  if (B == 0) {
+    // no tokens: grad_x is empty and grad_c is an empty sum
+    if (grad_c == nullptr) return RDFFT_OK;
+    if (!aligned16(grad_c)) return RDFFT_EALIGN;
+    return finish(cudaMemsetAsync(grad_c, 0, cb, reinterpret_cast<cudaStream_t>(stream)));
+  }
+  if (g == nullptr || c_hat == nullptr) return RDFFT_ENULL;
+  if (grad_c != nullptr && x == nullptr) return RDFFT_ENULL;
+  if (!aligned16(g) || !aligned16(c_hat) || (x && !aligned16(x)) || (grad_x && !aligned16(grad_x)) ||
+      (grad_c && !aligned16(grad_c)))
+    return RDFFT_EALIGN;
+  const size_t act = (size_t)B * D * (dtype == RDFFT_F32 ? 4 : 2);
+  if (overlap(grad_x, act, g, act) || overlap(grad_x, act, x, act) || overlap(grad_x, act, c_hat, cb) ||
+      overlap(grad_x, act, grad_c, cb) || overlap(grad_c, cb, g, act) || overlap(grad_c, cb, x, act) ||
+      overlap(grad_c, cb, c_hat, cb))
+    return RDFFT_EOVERLAP;
+  return kEnqueue;
+}
+
 }  // namespace
 
 extern "C" {
@@ -132,28 +164,49 @@ int circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p
 
 int circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
              int64_t B, int D, int p, int dtype, rdfft_stream_t stream) {
+  const int chk = bwd_args(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, stream);
+  if (chk != kEnqueue) return chk;
+  return finish(rdfft::launch_circ_bwd(g, x, c_hat, grad_x, grad_c, B, D, p, dtype,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int circ_bwd_workspace_size(int64_t B, int D, int p, int dtype, int with_grad_x, size_t* bytes) {
+  if (bytes == nullptr) return RDFFT_ENULL;
+  *bytes = 0;
   if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
   if (!layer_shape_ok(B, D, p)) return RDFFT_EINVAL;
-  if (grad_x == nullptr && grad_c == nullptr) return RDFFT_OK;
+  if (B == 0) return RDFFT_OK;
+  int slices = 0;
+  const cudaError_t e = rdfft::plan_circ_bwd(B, D, p, dtype, with_grad_x != 0, &slices);
+  if (e != cudaSuccess) return finish(e);
+  if (slices > 1) *bytes = (size_t)slices * gc_bytes(D, p);
+  return RDFFT_OK;
+}
+
+int circ_bwd_deterministic(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
+                           int64_t B, int D, int p, int dtype, void* workspace, size_t workspace_bytes,
+                           rdfft_stream_t stream) {
+  const int chk = bwd_args(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, stream);
+  if (chk != kEnqueue) return chk;
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const size_t cb = sizeof(float) * (size_t)(D / p) * (D / p) * p;
-  if (B == 0) {
-    // no tokens: grad_x is empty and grad_c is an empty sum
-    if (grad_c == nullptr) return RDFFT_OK;
-    if (!aligned16(grad_c)) return RDFFT_EALIGN;
-    return finish(cudaMemsetAsync(grad_c, 0, cb, s));
+  if (grad_c == nullptr) return finish(rdfft::launch_circ_bwd(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, s));
+  size_t need = 0;
+  const int rc = circ_bwd_workspace_size(B, D, p, dtype, grad_x != nullptr, &need);
+  if (rc != RDFFT_OK) return rc;
+  rdfft::GcSink sink;
+  if (need > 0) {
+    if (workspace == nullptr) return RDFFT_ENULL;
+    if (!aligned16(workspace)) return RDFFT_EALIGN;
+    if (workspace_bytes < need) return RDFFT_ESPACE;
+    const size_t act = (size_t)B * D * (dtype == RDFFT_F32 ? 4 : 2), cb = gc_bytes(D, p);
+    if (overlap(workspace, need, g, act) || overlap(workspace, need, x, act) ||
+        overlap(workspace, need, c_hat, cb) || overlap(workspace, need, grad_x, act) ||
+        overlap(workspace, need, grad_c, cb))
+      return RDFFT_EOVERLAP;
+    sink.partial = static_cast<float*>(workspace);
+    sink.partial_floats = (int64_t)(need / sizeof(float));
   }
-  if (g == nullptr || c_hat == nullptr) return RDFFT_ENULL;
-  if (grad_c != nullptr && x == nullptr) return RDFFT_ENULL;
-  if (!aligned16(g) || !aligned16(c_hat) || (x && !aligned16(x)) || (grad_x && !aligned16(grad_x)) ||
-      (grad_c && !aligned16(grad_c)))
-    return RDFFT_EALIGN;
-  const size_t act = (size_t)B * D * (dtype == RDFFT_F32 ? 4 : 2);
-  if (overlap(grad_x, act, g, act) || overlap(grad_x, act, x, act) || overlap(grad_x, act, c_hat, cb) ||
-      overlap(grad_x, act, grad_c, cb) || overlap(grad_c, cb, g, act) || overlap(grad_c, cb, x, act) ||
-      overlap(grad_c, cb, c_hat, cb))
-    return RDFFT_EOVERLAP;
-  return finish(rdfft::launch_circ_bwd(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, s));
+  return finish(rdfft::launch_circ_bwd(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, s, &sink));
 }
 
 int circ_fwd_tc(const void* x, const float* c_hat, void* y, int64_t B, int D, int p, int dtype,
@@ -191,6 +244,7 @@ const char* rdfft_strerror(int code) {
     case RDFFT_EDTYPE: return "dtype must be RDFFT_F32 (0) or RDFFT_BF16 (1)";
     case RDFFT_EOVERLAP: return "an output buffer overlaps an input buffer";
     case RDFFT_ETIMEOUT: return "a kernel's bounded wait for its data timed out; its rows were not transformed";
+    case RDFFT_ESPACE: return "the workspace is smaller than circ_bwd_workspace_size reports for this call";
     case RDFFT_ECUDA:
       snprintf(t_msg, sizeof(t_msg), "CUDA error while enqueuing: %s (%d)", cudaGetErrorString(t_last_cuda),
                (int)t_last_cuda);

@@ -23,6 +23,12 @@ inplace_spectrum (default False) chooses where c_hat lives during a call:
     (tests/test_layer_module_gpu.py). Use it where that drift is small against the
     optimizer's updates. While a call runs, c holds its spectrum: work on another
     stream must not read c until the call's stream has reached its end.
+
+The gradient of c is a sum over tokens. By default the token slices add into it with
+fp32 atomics, so its last bits can change from run to run; with deterministic=True, or
+whenever torch.use_deterministic_algorithms(True) is in force, the backward calls
+circ_bwd_deterministic instead (the slices summed in a fixed order through a workspace
+from torch's caching allocator).
 """
 from __future__ import annotations
 
@@ -35,9 +41,10 @@ from . import _binding as _b
 
 class _CirculantFn(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, x, c, p, inplace):
+    def forward(ctx, x, c, p, inplace, deterministic):
         ctx.p = p
         ctx.inplace = inplace
+        ctx.deterministic = deterministic or torch.are_deterministic_algorithms_enabled()
         shape = x.shape
         x2 = x.reshape(-1, shape[-1]).contiguous()
         with torch.no_grad():
@@ -62,17 +69,19 @@ class _CirculantFn(torch.autograd.Function):
                 c_hat = _b.rdfft_fwd(c.data, p)
             else:
                 c_hat = _b.circ_prepare(c.detach())
-            gx, gc = _b.circ_bwd(g2, x2, c_hat, p, need_grad_x=need_x, need_grad_c=need_c)
+            gx, gc = _b.circ_bwd(g2, x2, c_hat, p, need_grad_x=need_x, need_grad_c=need_c,
+                                 deterministic=ctx.deterministic)
             if ctx.inplace:
                 _b.rdfft_inv(c.data, p)
         if gx is not None:
             gx = gx.reshape(gy.shape)
-        return gx, gc, None, None
+        return gx, gc, None, None, None
 
 
-def block_circulant(x: torch.Tensor, c: torch.Tensor, p: int, inplace_spectrum: bool = False) -> torch.Tensor:
+def block_circulant(x: torch.Tensor, c: torch.Tensor, p: int, inplace_spectrum: bool = False,
+                    deterministic: bool = False) -> torch.Tensor:
     """y = W(c) x over the last dimension of x (bf16 or fp32); c: (q, q, p) fp32."""
-    return _CirculantFn.apply(x, c, p, inplace_spectrum)
+    return _CirculantFn.apply(x, c, p, inplace_spectrum, deterministic)
 
 
 class BlockCirculantLinear(torch.nn.Module):
@@ -84,7 +93,7 @@ class BlockCirculantLinear(torch.nn.Module):
     """
 
     def __init__(self, features: int, block: int, inplace_spectrum: bool = False, device=None,
-                 generator: torch.Generator | None = None):
+                 generator: torch.Generator | None = None, deterministic: bool = False):
         super().__init__()
         if block < 64 or block & (block - 1) or features % block:
             raise ValueError("block must be a power of two >= 64 dividing features")
@@ -94,9 +103,11 @@ class BlockCirculantLinear(torch.nn.Module):
         self.features = features
         self.block = block
         self.inplace_spectrum = inplace_spectrum
+        self.deterministic = deterministic
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:
-        return block_circulant(x, self.c, self.block, self.inplace_spectrum)
+        return block_circulant(x, self.c, self.block, self.inplace_spectrum, self.deterministic)
 
     def extra_repr(self) -> str:
-        return f"features={self.features}, block={self.block}, inplace_spectrum={self.inplace_spectrum}"
+        return (f"features={self.features}, block={self.block}, inplace_spectrum={self.inplace_spectrum}, "
+                f"deterministic={self.deterministic}")

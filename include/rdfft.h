@@ -42,6 +42,7 @@
 #ifndef RDFFT_H
 #define RDFFT_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -64,7 +65,8 @@ enum {
   RDFFT_EDTYPE = 4,   /* dtype is neither RDFFT_F32 nor RDFFT_BF16 */
   RDFFT_ECUDA = 5,    /* a CUDA call failed while enqueuing work */
   RDFFT_EOVERLAP = 6, /* an output buffer overlaps an input buffer it may not alias */
-  RDFFT_ETIMEOUT = 7  /* reported by rdfft_take_device_error(): a bounded device wait gave up */
+  RDFFT_ETIMEOUT = 7, /* reported by rdfft_take_device_error(): a bounded device wait gave up */
+  RDFFT_ESPACE = 8    /* the workspace is smaller than circ_bwd_workspace_size reports */
 };
 
 /* Largest feature size D accepted by circ_fwd / circ_bwd. */
@@ -188,11 +190,45 @@ int circ_fwd(const void* x, const float* c_hat, void* y, int64_t B, int D, int p
  *            matter. Must not overlap g, x or c_hat (RDFFT_EOVERLAP).
  * When the tokens are split over several CTAs, the grad_c sum over tokens is
  * accumulated with fp32 atomic adds into a zeroed buffer, so its last bits may differ
- * between runs. With a handful of tokens one CTA per block group sums them all and
- * stores the result, and grad_c is deterministic; grad_x and the forward always are.
+ * between runs (circ_bwd_deterministic below does not). With a handful of tokens one CTA
+ * per block group sums them all and stores the result, and grad_c is deterministic; grad_x
+ * and the forward always are.
  */
 int circ_bwd(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
              int64_t B, int D, int p, int dtype, rdfft_stream_t stream);
+
+/*
+ * circ_bwd_workspace_size -- device workspace, in bytes, that circ_bwd_deterministic needs
+ * for these sizes on the current device, with grad_c requested and grad_x too when
+ * with_grad_x != 0 (the two requests can take different kernels). 0 when the tokens fit
+ * one slice per block group, whose sums need no workspace. Otherwise slices x q x q x p x 4
+ * bytes, the slice count being what the grad_c kernel's grid uses for B tokens on this
+ * device's SM count (at most one slice per SM). Enqueues nothing; needs no GPU (without one
+ * it assumes 148 SMs).
+ *   bytes : written. NULL returns RDFFT_ENULL.
+ * Returns RDFFT_OK, RDFFT_EINVAL / RDFFT_EDTYPE as circ_bwd, or RDFFT_ECUDA.
+ */
+int circ_bwd_workspace_size(int64_t B, int D, int p, int dtype, int with_grad_x, size_t* bytes);
+
+/*
+ * circ_bwd_deterministic -- circ_bwd with a grad_c that is the same bit for bit from run to
+ * run on a given GPU model (the slice count follows the SM count). [notes] "Circulant matrix
+ * training adaptation", as circ_bwd; the sum over tokens is the same, only its order is
+ * fixed: each token slice stores its packed partial sum in the workspace (slice s at byte
+ * offset s q^2 p 4), and one more kernel adds the slices in order 0, 1, 2, ... into grad_c
+ * before the in-place rdIFFT. grad_x is computed exactly as by circ_bwd.
+ *   g, x, c_hat, grad_x, grad_c, B, D, p, dtype : as circ_bwd.
+ *   workspace       : device memory owned by the caller, at least circ_bwd_workspace_size
+ *                     bytes (same B, D, p, dtype, with_grad_x = grad_x != NULL), 16-byte
+ *                     aligned; overwritten, and may be NULL when that size is 0. Must not
+ *                     overlap any other argument (RDFFT_EOVERLAP).
+ *   workspace_bytes : its size; too small returns RDFFT_ESPACE before anything is enqueued.
+ * Costs one extra pass over the workspace (slices x q^2 p x 4 bytes written and read once).
+ * Calls that share a workspace must be ordered on one stream.
+ */
+int circ_bwd_deterministic(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
+                           int64_t B, int D, int p, int dtype, void* workspace, size_t workspace_bytes,
+                           rdfft_stream_t stream);
 
 /*
  * circ_fwd_tc, circ_bwd_x_tc -- the layer's forward and grad_x (as circ_fwd, and circ_bwd

@@ -13,7 +13,7 @@ from conftest import ROOT
 PKG = os.path.join(ROOT, "block_circulant_layers_b200")
 HEADER = os.path.join(ROOT, "include", "rdfft.h")
 
-OK, EINVAL, ENULL, EALIGN, EDTYPE, ECUDA, EOVERLAP, ETIMEOUT = range(8)
+OK, EINVAL, ENULL, EALIGN, EDTYPE, ECUDA, EOVERLAP, ETIMEOUT, ESPACE = range(9)
 F32, BF16 = 0, 1
 
 
@@ -34,6 +34,8 @@ def lib():
     L.circ_bwd.argtypes = [vp, vp, vp, vp, vp, i64, i, i, i, vp]
     L.circ_fwd_tc.argtypes = [vp, vp, vp, i64, i, i, i, vp]
     L.circ_bwd_x_tc.argtypes = [vp, vp, vp, i64, i, i, i, vp]
+    L.circ_bwd_workspace_size.argtypes = [i64, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
+    L.circ_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, i64, i, i, i, vp, ctypes.c_size_t, vp]
     L.rdfft_strerror.argtypes = [i]
     L.rdfft_strerror.restype = ctypes.c_char_p
     return L
@@ -48,7 +50,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("rdfft_fwd", "rdfft_inv", "rdfft_to_complex", "rdfft_from_complex", "rdfft2_fwd", "rdfft2_inv",
-              "circ_prepare", "circ_fwd", "circ_bwd", "circ_fwd_tc", "circ_bwd_x_tc", "rdfft_strerror",
+              "circ_prepare", "circ_fwd", "circ_bwd", "circ_fwd_tc", "circ_bwd_x_tc", "circ_bwd_workspace_size",
+              "circ_bwd_deterministic", "rdfft_strerror",
               "rdfft_version",
               "rdfft_take_device_error",
               "rdfft_selftest_wait_timeout"):
@@ -67,8 +70,9 @@ def test_library_exports_every_declared_symbol(lib):
 
 def test_version_and_messages(lib):
     assert lib.rdfft_version() >= 100
-    for code in range(8):
+    for code in range(9):
         assert lib.rdfft_strerror(code)
+    assert b"workspace" in lib.rdfft_strerror(ESPACE)
     assert b"unknown" in lib.rdfft_strerror(99)
 
 
@@ -137,6 +141,56 @@ def test_circ_argument_errors(lib):
     assert lib.circ_bwd(A, A, Bp, A, None, 4, D, p, BF16, None) == EOVERLAP        # grad_x == g
     assert lib.circ_bwd(A, A + (1 << 25), Bp, None, A, 4, D, p, BF16, None) == EOVERLAP
     assert lib.circ_bwd(A, A + (1 << 25), Bp, A + (1 << 26), None, 4, 4000, p, BF16, None) == EINVAL
+
+
+def workspace_size(lib, B, D, p, dtype=BF16, with_gx=1):
+    n = ctypes.c_size_t(12345)
+    rc = lib.circ_bwd_workspace_size(B, D, p, dtype, with_gx, ctypes.byref(n))
+    return rc, n.value
+
+
+def test_deterministic_backward_workspace_size(lib):
+    """The workspace query runs the launchers' own shape choice without a GPU (148 SMs
+    assumed): slices x q^2 p x 4 bytes, 0 for one slice, and the usual shape errors."""
+    assert lib.circ_bwd_workspace_size(4, 4096, 128, BF16, 1, None) == ENULL
+    assert workspace_size(lib, 4, 4000, 128) == (EINVAL, 0)
+    assert workspace_size(lib, 4, 4096, 32) == (EINVAL, 0)
+    assert workspace_size(lib, 4, 4096, 128, dtype=3) == (EDTYPE, 0)
+    assert workspace_size(lib, 0, 4096, 128) == (OK, 0)              # empty batch
+    assert workspace_size(lib, 1, 4096, 128) == (OK, 0)              # one slice stores grad_c
+    assert workspace_size(lib, 3, 4096, 512) == (OK, 0)
+    # D = 4096, p = 128, B = 256: 4 input-block groups x 32 slices of two 4-token tiles, both
+    # with grad_x (one kernel) and without (the grad_c kernel); 32 x 512 KiB
+    assert workspace_size(lib, 256, 4096, 128) == (OK, 32 * 32 * 32 * 128 * 4)
+    assert workspace_size(lib, 256, 4096, 128, with_gx=0) == (OK, 32 * 32 * 32 * 128 * 4)
+    # the adapter shape, D = 4096, p = 512, B = 4096: 147 slices of 7 tiles
+    assert workspace_size(lib, 4096, 4096, 512) == (OK, 147 * 8 * 8 * 512 * 4)
+    # one block, p = 4096, B = 4096, 2-token tiles: 147 slices
+    assert workspace_size(lib, 4096, 4096, 4096) == (OK, 147 * 4096 * 4)
+    for B in (1, 2, 5, 64, 255, 256, 1000, 4097):
+        for D, p in ((4096, 128), (4096, 512), (1024, 64), (2048, 1024), (8192, 4096)):
+            rc, n = workspace_size(lib, B, D, p)
+            q = D // p
+            assert rc == OK and n % (q * q * p * 4) == 0 and n // (q * q * p * 4) <= 148
+
+
+def test_deterministic_backward_argument_errors(lib):
+    """Checked before anything is enqueued: the circ_bwd checks, then the workspace's."""
+    B, D, p = 256, 4096, 128
+    need = 32 * 32 * 32 * 128 * 4                     # 16 MiB (see the test above)
+    g, x, gx = A, A + (1 << 22), A + (1 << 23)        # 2 MiB bf16 activations each
+    ch, gc, ws = Bp, Bp + (1 << 20), Bp + (1 << 24)   # c_hat, grad_c: 512 KiB each
+    f = lib.circ_bwd_deterministic
+    assert f(g, x, ch, None, None, B, D, p, BF16, None, 0, None) == OK         # nothing asked
+    assert f(g, x, ch, gx, gc, B, 4000, p, BF16, ws, need, None) == EINVAL
+    assert f(g, x, ch, gx, gc, B, D, p, 7, ws, need, None) == EDTYPE
+    assert f(None, x, ch, gx, gc, B, D, p, BF16, ws, need, None) == ENULL
+    assert f(g, x, ch, g, gc, B, D, p, BF16, ws, need, None) == EOVERLAP       # grad_x == g
+    assert f(g, x, ch, gx, gc, B, D, p, BF16, None, need, None) == ENULL       # workspace needed
+    assert f(g, x, ch, gx, gc, B, D, p, BF16, ws + 4, need, None) == EALIGN
+    assert f(g, x, ch, gx, gc, B, D, p, BF16, ws, need - 16, None) == ESPACE
+    assert f(g, x, ch, gx, gc, B, D, p, BF16, g, need, None) == EOVERLAP       # workspace over g
+    assert f(g, x, ch, gx, gc, B, D, p, BF16, gc - 4096, need, None) == EOVERLAP
 
 
 def test_circ_prepare_argument_errors(lib):
