@@ -33,9 +33,10 @@ lib.circ_fwd_tc.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_bwd_x_tc.argtypes = [_vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 lib.circ_bwd_workspace_size.argtypes = [_i64, _int, _int, _int, _int, ctypes.POINTER(ctypes.c_size_t)]
 lib.circ_bwd_deterministic.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _vp, ctypes.c_size_t, _vp]
+lib.circ_bwd_deterministic_noalloc.argtypes = [_vp, _vp, _vp, _vp, _vp, _i64, _int, _int, _int, _vp]
 for _f in (lib.rdfft_fwd, lib.rdfft_inv, lib.rdfft_to_complex, lib.rdfft_from_complex, lib.rdfft2_fwd,
            lib.rdfft2_inv, lib.circ_prepare, lib.circ_fwd, lib.circ_bwd, lib.circ_fwd_tc, lib.circ_bwd_x_tc,
-           lib.circ_bwd_workspace_size, lib.circ_bwd_deterministic):
+           lib.circ_bwd_workspace_size, lib.circ_bwd_deterministic, lib.circ_bwd_deterministic_noalloc):
     _f.restype = _int
 lib.rdfft_strerror.argtypes = [_int]
 lib.rdfft_strerror.restype = ctypes.c_char_p

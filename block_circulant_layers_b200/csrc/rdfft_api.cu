@@ -5,6 +5,8 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <mutex>
+
 #include "rdfft.h"
 #include "internal.h"
 
@@ -111,6 +113,33 @@ int bwd_args(const void* g, const void* x, const float* c_hat, void* grad_x, flo
   return kEnqueue;
 }
 
+// Scratch of circ_bwd_deterministic_noalloc: its per-slice grad_c sums live here instead
+// of in caller memory. Every device that loads the library holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = RDFFT_NOALLOC_SCRATCH_BYTES;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of g_noalloc_scratch on the current device. In host code the array's name
+// is only a stand-in, so the address is looked up with cudaGetSymbolAddress, once per
+// device with that device current, and kept (no host or device allocation).
+constexpr int kMaxDevices = 64;
+cudaError_t noalloc_scratch(float** ptr) {
+  static std::mutex mu;
+  static float* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<float*>(p);
+  }
+  *ptr = addr[dev];
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -209,6 +238,27 @@ int circ_bwd_deterministic(const void* g, const void* x, const float* c_hat, voi
   return finish(rdfft::launch_circ_bwd(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, s, &sink));
 }
 
+int circ_bwd_deterministic_noalloc(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
+                                   int64_t B, int D, int p, int dtype, rdfft_stream_t stream) {
+  const int chk = bwd_args(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, stream);
+  if (chk != kEnqueue) return chk;
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (grad_c == nullptr) return finish(rdfft::launch_circ_bwd(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, s));
+  size_t need = 0;
+  const int rc = circ_bwd_workspace_size(B, D, p, dtype, grad_x != nullptr, &need);
+  if (rc != RDFFT_OK) return rc;
+  if (need > kNoAllocScratchBytes) return RDFFT_ESPACE;
+  rdfft::GcSink sink;
+  if (need > 0) {
+    float* scratch = nullptr;
+    const cudaError_t e = noalloc_scratch(&scratch);
+    if (e != cudaSuccess) return finish(e);
+    sink.partial = scratch;
+    sink.partial_floats = (int64_t)(need / sizeof(float));
+  }
+  return finish(rdfft::launch_circ_bwd(g, x, c_hat, grad_x, grad_c, B, D, p, dtype, s, &sink));
+}
+
 int circ_fwd_tc(const void* x, const float* c_hat, void* y, int64_t B, int D, int p, int dtype,
                 rdfft_stream_t stream) {
   if (!dtype_ok(dtype)) return RDFFT_EDTYPE;
@@ -244,7 +294,9 @@ const char* rdfft_strerror(int code) {
     case RDFFT_EDTYPE: return "dtype must be RDFFT_F32 (0) or RDFFT_BF16 (1)";
     case RDFFT_EOVERLAP: return "an output buffer overlaps an input buffer";
     case RDFFT_ETIMEOUT: return "a kernel's bounded wait for its data timed out; its rows were not transformed";
-    case RDFFT_ESPACE: return "the workspace is smaller than circ_bwd_workspace_size reports for this call";
+    case RDFFT_ESPACE:
+      return "the workspace is smaller than circ_bwd_workspace_size reports for this call (for "
+             "circ_bwd_deterministic_noalloc: the call needs more than its built-in 16 MiB of scratch)";
     case RDFFT_ECUDA:
       snprintf(t_msg, sizeof(t_msg), "CUDA error while enqueuing: %s (%d)", cudaGetErrorString(t_last_cuda),
                (int)t_last_cuda);

@@ -231,6 +231,30 @@ int circ_bwd_deterministic(const void* g, const void* x, const float* c_hat, voi
                            rdfft_stream_t stream);
 
 /*
+ * circ_bwd_deterministic_noalloc -- circ_bwd_deterministic for callers that cannot allocate
+ * device memory: the same kernels and the same result bit for bit, with the workspace taken
+ * from a scratch array built into the library instead of from the caller. The paper has no
+ * counterpart; this is an interface convenience.
+ *   g, x, c_hat, grad_x, grad_c, B, D, p, dtype : as circ_bwd.
+ * Scratch: a file-scope device array of 16 MiB (RDFFT_NOALLOC_SCRATCH_BYTES) that every GPU
+ * loading the library holds until the process exits. A call whose workspace
+ * (circ_bwd_workspace_size) would exceed it returns RDFFT_ESPACE before enqueuing anything.
+ * At 148 SMs, D = 4096, p = 128, B = 256 needs 16 MiB and fits; D = 4096, p = 512, B = 4096
+ * needs 18.4 MiB and is refused; no shape needs more than 20 MiB. Nothing in it has to
+ * start at zero: each call stores every element of the slices it then reads.
+ * Set-up: the first call on each device (with that device current) looks up the array's
+ * device address (cudaGetSymbolAddress) and keeps it; make that first call before any
+ * stream capture on the device. Later calls do no set-up.
+ * Sharing: every call on a device uses the same array, which keeps the last call's
+ * contents. Calls that overlap on the GPU (different streams without ordering between
+ * them, or several host threads) race on it and may return wrong grad_c; order them on
+ * one stream. Allocates nothing: no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define RDFFT_NOALLOC_SCRATCH_BYTES (16u << 20)
+int circ_bwd_deterministic_noalloc(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
+                                   int64_t B, int D, int p, int dtype, rdfft_stream_t stream);
+
+/*
  * circ_fwd_tc, circ_bwd_x_tc -- the layer's forward and grad_x (as circ_fwd, and circ_bwd
  * with grad_c = NULL) with the per-frequency-bin contraction on the fifth-generation
  * tensor cores: tcgen05.mma of kind::tf32 with fp32 accumulation in tensor memory.

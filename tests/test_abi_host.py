@@ -36,6 +36,7 @@ def lib():
     L.circ_bwd_x_tc.argtypes = [vp, vp, vp, i64, i, i, i, vp]
     L.circ_bwd_workspace_size.argtypes = [i64, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
     L.circ_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, i64, i, i, i, vp, ctypes.c_size_t, vp]
+    L.circ_bwd_deterministic_noalloc.argtypes = [vp, vp, vp, vp, vp, i64, i, i, i, vp]
     L.rdfft_strerror.argtypes = [i]
     L.rdfft_strerror.restype = ctypes.c_char_p
     return L
@@ -51,7 +52,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for n in ("rdfft_fwd", "rdfft_inv", "rdfft_to_complex", "rdfft_from_complex", "rdfft2_fwd", "rdfft2_inv",
               "circ_prepare", "circ_fwd", "circ_bwd", "circ_fwd_tc", "circ_bwd_x_tc", "circ_bwd_workspace_size",
-              "circ_bwd_deterministic", "rdfft_strerror",
+              "circ_bwd_deterministic", "circ_bwd_deterministic_noalloc", "rdfft_strerror",
               "rdfft_version",
               "rdfft_take_device_error",
               "rdfft_selftest_wait_timeout"):
@@ -191,6 +192,35 @@ def test_deterministic_backward_argument_errors(lib):
     assert f(g, x, ch, gx, gc, B, D, p, BF16, ws, need - 16, None) == ESPACE
     assert f(g, x, ch, gx, gc, B, D, p, BF16, g, need, None) == EOVERLAP       # workspace over g
     assert f(g, x, ch, gx, gc, B, D, p, BF16, gc - 4096, need, None) == EOVERLAP
+
+
+def test_noalloc_backward_argument_errors(lib):
+    """The built-in-scratch variant checks like circ_bwd and refuses, before enqueuing
+    anything, a call whose workspace would exceed its 16 MiB."""
+    f = lib.circ_bwd_deterministic_noalloc
+    B, D, p = 256, 4096, 128
+    g, x, gx = A, A + (1 << 22), A + (1 << 23)
+    ch, gc = Bp, Bp + (1 << 20)
+    assert f(g, x, ch, None, None, B, D, p, BF16, None) == OK                 # nothing asked
+    assert f(g, x, ch, gx, gc, B, 4000, p, BF16, None) == EINVAL
+    assert f(g, x, ch, gx, gc, B, D, p, 9, None) == EDTYPE
+    assert f(g, None, ch, gx, gc, B, D, p, BF16, None) == ENULL
+    assert f(g, x, ch, gx + 2, gc, B, D, p, BF16, None) == EALIGN
+    assert f(g, x, ch, gc, gc, B, D, p, BF16, None) == EOVERLAP
+    # D = 8192, p = 64 (q = 128: 4 MiB of grad_c per token slice), B = 4096: 5 slices, 20 MiB;
+    # the adapter shape D = 4096, p = 512, B = 4096: 147 slices, 18.4 MiB
+    for B, D, p in ((4096, 8192, 64), (4096, 4096, 512)):
+        rc, need = workspace_size(lib, B, D, p)
+        assert rc == OK and need > (16 << 20)
+        q = D // p
+        g, x, gx = A, A + (1 << 27), A + (1 << 28)      # up to 64 MiB bf16 activations each
+        ch, gc = Bp, Bp + (1 << 23)                     # up to 4 MiB c_hat / grad_c
+        assert f(g, x, ch, gx, gc, B, D, p, BF16, None) == ESPACE
+    # the same tokens without grad_x take the grad_c kernel: one input-block group of 147
+    # slices, 18.4 MiB
+    rc, need = workspace_size(lib, 4096, 4096, 512, with_gx=0)
+    assert rc == OK and need > (16 << 20)
+    assert f(A, A + (1 << 27), Bp, None, Bp + (1 << 23), 4096, 4096, 512, BF16, None) == ESPACE
 
 
 def test_circ_prepare_argument_errors(lib):
