@@ -182,19 +182,24 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
       return SM::STG ? stage + SM::STAGE_G + (size_t)(t * QJ + jl) * P
                      : x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P;
     };
+    // only the rows of the tile's ntok tokens are transformed: the r-th is g row r for
+    // r < ntok q, then x row XR + (r - ntok q), so a partial last tile takes fewer rounds
+    // of rows (the rows of absent tokens keep stale values that nothing stores)
+    const int ngr = ntok * q, nrows = ntok * (q + QJ);
+    auto rowmap = [=](int r) { return r < ngr ? r : XR + (r - ngr); };
     {
       constexpr int TPR = G::TPR, RPR = NT / TPR;
       const int v = threadIdx.x % TPR;
-      for (int r = threadIdx.x / TPR; r < XR + TT * QJ; r += RPR) {
-        const T* row = src(r);
-        fwd_pass0<G, T>(tile, r, v, row, row != nullptr);
+      for (int rr = threadIdx.x / TPR; rr < nrows; rr += RPR) {
+        const int r = rowmap(rr);
+        fwd_pass0<G, T>(tile, r, v, src(r), true);
       }
     }
     if constexpr (SM::STG) {
       __syncthreads();                               // the staged rows are read: fetch the next tile's
       if (threadIdx.x == 0 && tok0 + TT < tend) fill(tok0 + TT);
     }
-    fft_rows_rest<P, NT, T, 1>(tile, XR + TT * QJ, src);
+    fft_rows_rest_mapped<P, NT, T, 1>(tile, nrows, rowmap);
     __syncthreads();
 
     // 2. cross-spectrum: S_ij += G_i conj(X_j) over the tile's tokens, from and back to
@@ -331,7 +336,9 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
           const f2 cr = f2_bc(ch[cb]), ci = f2_bc(ch[cb + 1]);
 #pragma unroll
           for (int v = 0; v < TT / 2; ++v) {
-            // rows of tokens beyond ntok hold zeros (their transforms read no input)
+            // a pair past the tile's tokens is skipped; in a pair whose second token is absent,
+            // that lane works on a stale row and is never stored (the lanes are independent)
+            if (2 * v >= ntok) break;
             const int rb0 = G::row_base(2 * v * Q + i), rb1 = G::row_base((2 * v + 1) * Q + i);
             const float vr0 = tile[rb0 + xkr], vi0 = tile[rb0 + xki];
             const float vr1 = tile[rb1 + xkr], vi1 = tile[rb1 + xki];
@@ -358,9 +365,9 @@ k_circ_bwd_fused(const T* __restrict__ g, const T* __restrict__ x, const float* 
     }
     __syncthreads();
     // 4. rdIFFT (Hartley form) of the grad_x rows straight to HBM
-    ifft_rows_mirrored<P, NT, T>(tile + G::row_base(XR), TT * QJ, [&](int r) -> T* {
+    ifft_rows_mirrored<P, NT, T>(tile + G::row_base(XR), ntok * QJ, [&](int r) -> T* {
       const int t = r / QJ, jl = r - t * QJ;
-      return t < ntok ? grad_x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P : nullptr;
+      return grad_x + (tok0 + t) * (int64_t)D + (int64_t)(j0 + jl) * P;
     });
   }
 

@@ -40,18 +40,25 @@ namespace rdfft {
 // accumulators.
 
 // ------------------------------------------------------------- tile row passes
-// Orbit pass K (tile -> tile) over tile rows [0, NR): every thread runs the generic
-// orbits of its rows, then the NR * NB merged orbits are spread one per thread.
-template <int P, int NT, int K, bool INV, typename T>
-__device__ __forceinline__ void tile_orbit_pass(float* tile, int NR) {
+// Orbit pass K (tile -> tile) over NR rows of the tile, the r-th being tile row rowmap(r)
+// (consecutive rows, [0, NR), for tile_orbit_pass): every thread runs the generic orbits of
+// its rows, then the NR * NB merged orbits are spread one per thread. Rows that share a
+// warp must map to consecutive tile rows in aligned groups of RW.
+template <int P, int NT, int K, bool INV, typename T, typename RowMap>
+__device__ __forceinline__ void tile_orbit_pass_mapped(float* tile, int NR, RowMap rowmap) {
   using G = LayerGeo<P>;
   constexpr int TPR = G::TPR, RPR = NT / TPR;
   constexpr int NB = PassShape<G, K>::NB;
   const int v = threadIdx.x % TPR;
   for (int r = threadIdx.x / TPR; r < NR; r += RPR)
-    generic_pass<G, K, INV, 0, 0>(tile, r, v, (T*)nullptr, false);
+    generic_pass<G, K, INV, 0, 0>(tile, rowmap(r), v, (T*)nullptr, false);
   for (int mu = threadIdx.x; mu < NR * NB; mu += NT)
-    merged_orbit<G, K, INV, 0, 0>(tile, mu / NB, mu % NB, (T*)nullptr, false);
+    merged_orbit<G, K, INV, 0, 0>(tile, rowmap(mu / NB), mu % NB, (T*)nullptr, false);
+}
+
+template <int P, int NT, int K, bool INV, typename T>
+__device__ __forceinline__ void tile_orbit_pass(float* tile, int NR) {
+  tile_orbit_pass_mapped<P, NT, K, INV, T>(tile, NR, [](int r) { return r; });
 }
 
 // Forward rdFFT of tile rows [0, NR): row r reads its input from src(r) (nullptr
@@ -62,6 +69,17 @@ __device__ __forceinline__ void fft_rows_rest(float* tile, int NR, SrcFn src) {
     __syncthreads();
     tile_orbit_pass<P, NT, K, false, T>(tile, NR);
     fft_rows_rest<P, NT, T, K + 1>(tile, NR, src);
+  }
+}
+
+// Passes K.. of the forward rdFFT of NR rows mapped to tile rows by rowmap (see
+// tile_orbit_pass_mapped); pass 0 is the caller's.
+template <int P, int NT, typename T, int K, typename RowMap>
+__device__ __forceinline__ void fft_rows_rest_mapped(float* tile, int NR, RowMap rowmap) {
+  if constexpr (K < LayerGeo<P>::NPASS) {
+    __syncthreads();
+    tile_orbit_pass_mapped<P, NT, K, false, T>(tile, NR, rowmap);
+    fft_rows_rest_mapped<P, NT, T, K + 1>(tile, NR, rowmap);
   }
 }
 
