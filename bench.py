@@ -958,6 +958,10 @@ PROFILE_CASES = {
     "circ_bwd_d4096_p512_b4096": ("circ", (4096, 4096, 512, "bwd")),
     "circ_bwd_d4096_p128_b256": ("circ", (256, 4096, 128, "bwd")),
     "circ_step_d4096_p128_b1": ("circ_step", (1, 4096, 128)),
+    "circ_step_d4096_p128_b256": ("circ_step", (256, 4096, 128)),
+    "circ_step_d1024_p1024_b256": ("circ_step", (256, 1024, 1024)),
+    "circ_bwd_det_d4096_p128_b256": ("circ", (256, 4096, 128, "bwd_det")),
+    "circ_bwd_det_d4096_p512_b4096": ("circ", (4096, 4096, 512, "bwd_det")),
     "step_round": ("step_round", ()),
 }
 
@@ -1027,6 +1031,7 @@ def run_profile_case(name: str) -> int:
         g = torch.randn(B, D, device=dev, generator=gen).to(torch.bfloat16)
         y = torch.empty_like(x)
         gc = torch.empty_like(c)
+        ws = torch.empty(max(16, rd.circ_bwd_workspace_size(B, D, p, torch.bfloat16)), dtype=torch.uint8, device=dev)
         for _ in range(4):
             if d == "fwd":
                 rd.circ_fwd(x, ch, p, y=y)
@@ -1034,6 +1039,8 @@ def run_profile_case(name: str) -> int:
                 rd.circ_fwd_tc(x, ch, p, y=y)
             elif d == "bwd":
                 rd.circ_bwd(g, x, ch, p, grad_x=y, grad_c=gc)
+            elif d == "bwd_det":
+                rd.circ_bwd(g, x, ch, p, grad_x=y, grad_c=gc, deterministic=True, workspace=ws)
             elif d == "bwdx":
                 rd.circ_bwd(g, x, ch, p, grad_x=y, need_grad_c=False)
             else:
