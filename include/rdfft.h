@@ -224,7 +224,9 @@ int circ_bwd_workspace_size(int64_t B, int D, int p, int dtype, int with_grad_x,
  *                     overlap any other argument (RDFFT_EOVERLAP).
  *   workspace_bytes : its size; too small returns RDFFT_ESPACE before anything is enqueued.
  * Costs one extra pass over the workspace (slices x q^2 p x 4 bytes written and read once).
- * Calls that share a workspace must be ordered on one stream.
+ * Calls that share a workspace must be ordered on one stream. As with circ_bwd, a CTA whose
+ * bounded wait gives up (rdfft_take_device_error then returns RDFFT_ETIMEOUT) leaves its part
+ * unwritten, and grad_c is then wrong.
  */
 int circ_bwd_deterministic(const void* g, const void* x, const float* c_hat, void* grad_x, float* grad_c,
                            int64_t B, int D, int p, int dtype, void* workspace, size_t workspace_bytes,
