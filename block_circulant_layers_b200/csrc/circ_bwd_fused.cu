@@ -20,8 +20,10 @@
 // contraction. Beside it each thread keeps the c_hat values of its grad_x slots (one
 // bin, NS output blocks, all q summed blocks: 64 floats at p = 512), read from HBM once
 // per CTA instead of once per tile. At the end each CTA adds its part into grad_c (fp32
-// red.add into a zeroed grad_c; a plain store when one CTA per group covers all tokens), and
-// the caller's stream runs the in-place rdIFFT of grad_c's q^2 rows after, as circ_bwd does.
+// red.add into a zeroed grad_c; a plain store when one CTA per group covers all tokens, or
+// into its slice's part of the workspace in the deterministic mode), and the caller's
+// stream runs the in-place rdIFFT of grad_c's q^2 rows after, as circ_bwd does. Layers
+// of one or two blocks take k_circ_bwd_small below, with the cross-spectrum in registers.
 #include <cuda_runtime.h>
 
 #include "bulk_copy.cuh"

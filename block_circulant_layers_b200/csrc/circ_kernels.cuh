@@ -19,9 +19,12 @@
 //  * k_circ_gc (grad_c): a persistent CTA owns a group of QJ input blocks j and a
 //    slice of the tokens; it keeps its part of the packed cross-spectrum
 //    S_ij = sum_b G_i conj(X_j) in registers across all its token tiles and adds it
-//    into grad_c once (fp32 red.add; a plain store when a single token slice covers
-//    all tokens, and grad_c then needs no zeroing). grad_c is rdIFFT'd in place
-//    after, so the output buffer is the only global storage used.
+//    into grad_c once (fp32 red.add into a grad_c zeroed by k_zero_f4; a plain store
+//    when a single token slice covers all tokens, and grad_c then needs no zeroing).
+//    grad_c is rdIFFT'd in place after, so the output buffer is the only global
+//    storage used. In the deterministic mode (circ_bwd_deterministic) each slice
+//    instead stores its sums into its own q x q x p part of a caller workspace, and
+//    the slices are summed in a fixed order (k_sum_slices, circ_launch.cu).
 //  * For some shapes circ_bwd with both gradients runs one kernel instead of k_circ_x
 //    (grad_x) and k_circ_gc (circ_bwd_fused.cu).
 #pragma once
