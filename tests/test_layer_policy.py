@@ -106,3 +106,21 @@ def test_grad_c_token_slices(emu):
             # a single slice (grad_c stored, no zeroing) exactly when one tile or one CTA
             # per group is all there is
             assert (s == 1) == (ntiles == 1 or -(-N_SM // njgroups) == 1)
+
+
+def test_forward_token_tiles(emu):
+    """4-token tiles unless their grid would split a token's output blocks over CTAs."""
+    emu.rdfft_layer_x_tokens.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    # D = 4096, p = 512 (q = 8, 8 output blocks per CTA): 64 groups of 4 tokens would need the
+    # output blocks split in two; 2-token tiles give 128 CTAs of all 8
+    assert emu.rdfft_layer_x_tokens(256, 8, 8, N_SM) == 2
+    assert emu.rdfft_layer_x_tokens(512, 8, 8, N_SM) == 4
+    assert emu.rdfft_layer_x_tokens(4096, 8, 8, N_SM) == 4
+    # D = 4096, p = 256 (q = 16): two output-block groups of 8 either way
+    assert emu.rdfft_layer_x_tokens(256, 16, 8, N_SM) == 4
+    for q in (1, 2, 4, 8, 16, 32, 64, 128):
+        for B in (256, 300, 512, 1024, 4096):
+            tt = emu.rdfft_layer_x_tokens(B, q, 8, N_SM)
+            assert tt in (2, 4)
+            qi_full = emu.rdfft_layer_qi(q, 8, 1 << 30, N_SM)
+            assert (tt == 4) == (emu.rdfft_layer_qi(q, 8, -(-B // 4), N_SM) == qi_full)
