@@ -682,8 +682,8 @@ static cudaError_t launch_x_cfg(const void* in, const float* chat, void* out, in
 
 // Launch policy (at most 32 complex accumulators per thread, NS * TT <= 32):
 //  p <= 512 : 256 threads, up to 8 output blocks per CTA (16 at p = 128 from B = 256),
-//             1/2/4 tokens per CTA by B (4 only when that grid still covers most SMs,
-//             layer_x_tokens);
+//             up to 4 tokens per CTA from B = 256, 2 from B = 32, fewer when the grid would
+//             otherwise split a token's output blocks over CTAs (layer_x_tokens);
 //  p >= 1024: 128 threads, one token per CTA (4 for the q = 1, p = 1024 layer; one
 //             output block per CTA for q = 1 at p >= 2048).
 template <int P, typename T, bool BWDX>
@@ -701,9 +701,12 @@ static cudaError_t launch_x_p(const void* in, const float* chat, void* out, int6
       if (B >= 256 && q >= 16) return launch_x_cfg<P, T, 512, 2, 4, BWDX>(in, chat, out, B, q, s);
       if (B >= 256) return launch_x_cfg<P, T, NT, 4, 2 * NS, BWDX>(in, chat, out, B, q, s);
     }
-    if (B >= 256 && NS * 4 <= 32 && layer_x_tokens(B, q, NS * NT / (P / 2), num_sms()) == 4)
-      return launch_x_cfg<P, T, NT, 4, NS, BWDX>(in, chat, out, B, q, s);
-    if (B >= 32) return launch_x_cfg<P, T, NT, 2, NS, BWDX>(in, chat, out, B, q, s);
+    const int tt_max = (B >= 256 && NS * 4 <= 32) ? 4 : (B >= 32 ? 2 : 1);
+    const int tt = layer_x_tokens(B, q, NS * NT / (P / 2), num_sms(), tt_max);
+    if constexpr (NS * 4 <= 32) {
+      if (tt == 4) return launch_x_cfg<P, T, NT, 4, NS, BWDX>(in, chat, out, B, q, s);
+    }
+    if (tt == 2) return launch_x_cfg<P, T, NT, 2, NS, BWDX>(in, chat, out, B, q, s);
     return launch_x_cfg<P, T, NT, 1, NS, BWDX>(in, chat, out, B, q, s);
   } else {
     constexpr int NT = 128;

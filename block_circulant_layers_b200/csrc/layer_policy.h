@@ -24,15 +24,18 @@ inline int layer_qi(int q, int qi_max, int64_t gx, int n_sm) {
   return qi;
 }
 
-// Tokens per CTA of the forward / grad_x kernel for p <= 512 from 256 tokens on: 4 (each
-// c_hat value read serves four tokens), unless the grid of 4-token CTAs is so small that
-// layer_qi would split the output blocks over several CTAs, each transforming the same input
-// rows again; then 2, whose grid of twice the token groups keeps every output block of a
-// token in one CTA (D=4096 p=512 B=256: 9.6 against 11.5 us; D=2048 p=512 and D=1024
-// p=256 at B=256: 6.6 against 7.7 and 5.5 against 6.0 us).
-inline int layer_x_tokens(int64_t B, int q, int qi_max, int n_sm) {
-  const int64_t gx = (B + 3) / 4;
-  return layer_qi(q, qi_max, gx, n_sm) == largest_divisor_leq(q, qi_max) ? 4 : 2;
+// Tokens per CTA of the forward / grad_x kernel for p <= 512: the largest of tt_max, 2, 1
+// whose grid keeps all of a token's output blocks in one CTA, i.e. for which layer_qi does
+// not split the output blocks over several CTAs (each of which would transform the same input
+// rows again); 1 when every tile size would split them. More tokens per CTA let each c_hat
+// value read serve more tokens, so the split is the only reason to take fewer (forward at
+// D=4096 p=512: B=256 9.6 against 11.5 us, B=64 6.8 against 8.2; D=4096 p=256 B=32 6.5
+// against 8.2; D=2048 p=512 B=128 5.8 against 6.6).
+inline int layer_x_tokens(int64_t B, int q, int qi_max, int n_sm, int tt_max) {
+  const int full = largest_divisor_leq(q, qi_max);
+  for (int tt = tt_max; tt > 1; tt /= 2)
+    if (layer_qi(q, qi_max, (B + tt - 1) / tt, n_sm) == full) return tt;
+  return 1;
 }
 
 // Input blocks per grad_c CTA group: a divisor of q, at most 8, with at most

@@ -109,18 +109,26 @@ def test_grad_c_token_slices(emu):
 
 
 def test_forward_token_tiles(emu):
-    """4-token tiles unless their grid would split a token's output blocks over CTAs."""
-    emu.rdfft_layer_x_tokens.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    """The largest token tile whose grid keeps a token's output blocks in one CTA."""
+    f = emu.rdfft_layer_x_tokens
+    f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int]
     # D = 4096, p = 512 (q = 8, 8 output blocks per CTA): 64 groups of 4 tokens would need the
     # output blocks split in two; 2-token tiles give 128 CTAs of all 8
-    assert emu.rdfft_layer_x_tokens(256, 8, 8, N_SM) == 2
-    assert emu.rdfft_layer_x_tokens(512, 8, 8, N_SM) == 4
-    assert emu.rdfft_layer_x_tokens(4096, 8, 8, N_SM) == 4
-    # D = 4096, p = 256 (q = 16): two output-block groups of 8 either way
-    assert emu.rdfft_layer_x_tokens(256, 16, 8, N_SM) == 4
+    assert f(256, 8, 8, N_SM, 4) == 2
+    assert f(512, 8, 8, N_SM, 4) == 4
+    assert f(4096, 8, 8, N_SM, 4) == 4
+    assert f(64, 8, 8, N_SM, 2) == 1
+    # D = 4096, p = 256 (q = 16): two output-block groups of 8 at B = 256 either way
+    assert f(256, 16, 8, N_SM, 4) == 4
     for q in (1, 2, 4, 8, 16, 32, 64, 128):
-        for B in (256, 300, 512, 1024, 4096):
-            tt = emu.rdfft_layer_x_tokens(B, q, 8, N_SM)
-            assert tt in (2, 4)
-            qi_full = emu.rdfft_layer_qi(q, 8, 1 << 30, N_SM)
-            assert (tt == 4) == (emu.rdfft_layer_qi(q, 8, -(-B // 4), N_SM) == qi_full)
+        full = emu.rdfft_layer_qi(q, 8, 1 << 30, N_SM)
+        for B in (1, 5, 32, 64, 200, 256, 300, 512, 1024, 4096):
+            for tt_max in (1, 2, 4):
+                tt = f(B, q, 8, N_SM, tt_max)
+                assert tt in (1, 2, 4) and tt <= tt_max
+                if tt > 1:                   # the chosen tile keeps the output blocks whole
+                    assert emu.rdfft_layer_qi(q, 8, -(-B // tt), N_SM) == full
+                if tt < tt_max:              # and every larger one would split them
+                    for t2 in (2 * tt, 4 * tt):
+                        if t2 <= tt_max:
+                            assert emu.rdfft_layer_qi(q, 8, -(-B // t2), N_SM) != full
