@@ -592,9 +592,20 @@ cudaError_t fused_t(const void* g, const void* x, const float* chat, void* grad_
       default: return cudaErrorInvalidValue;
     }
   }
-  if (p == 128 && q == 32) return run_fused<128, 32, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s, sink);
-  if (p == 512 && q == 8) return run_fused<512, 8, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s, sink);
-  if (p == 1024 && q == 4) return run_fused<1024, 4, 4, T, 2, 4, 4>(g, x, chat, grad_x, grad_c, B, s, sink);
+  // tiles of 4 tokens (2 at p = 1024), or half that while all CTAs hold one tile in one wave
+  const int nsm = num_sms();
+  if (p == 128 && q == 32) {
+    if (layer_fused_small_tiles(B, 2, 4, nsm)) return run_fused<128, 32, 8, T, 2, 4, 8>(g, x, chat, grad_x, grad_c, B, s, sink);
+    return run_fused<128, 32, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s, sink);
+  }
+  if (p == 512 && q == 8) {
+    if (layer_fused_small_tiles(B, 2, 1, nsm)) return run_fused<512, 8, 8, T, 2, 4, 8>(g, x, chat, grad_x, grad_c, B, s, sink);
+    return run_fused<512, 8, 8, T, 4, 4, 8>(g, x, chat, grad_x, grad_c, B, s, sink);
+  }
+  if (p == 1024 && q == 4) {
+    if (layer_fused_small_tiles(B, 1, 1, nsm)) return run_fused<1024, 4, 4, T, 1, 4, 4>(g, x, chat, grad_x, grad_c, B, s, sink);
+    return run_fused<1024, 4, 4, T, 2, 4, 4>(g, x, chat, grad_x, grad_c, B, s, sink);
+  }
   return cudaErrorInvalidValue;
 }
 
@@ -608,16 +619,17 @@ cudaError_t take_fused_device_error(unsigned int* flags) {
   return e;
 }
 
-// p = 128 (q = 32) from 64 tokens on (backward at D = 4096: 22.9 against 26.1 us at B = 64,
-// 25.0 against 31.8 at B = 128); below, the two kernels, whose grids adapt to a handful of
-// tokens, are faster (17.9 against 19.6 us at B = 1)
+// p = 128 (q = 32) at every batch size (backward at D = 4096 with 2-token tiles: 13.8 against
+// 14.7 us for the two kernels at B = 1, 16.7 against 19.7 at B = 4, 16.7 against 21.3 at
+// B = 12; with 4-token tiles 24.0 against 31.8 at B = 128)
 // One or two blocks (D = p or 2 p) from p = 512 on, at every batch size (backward at D = p =
 // 4096: 15.0 against 17.3 us at B = 1, 15.4 against 21.7 at B = 256, 115.8 against 188.0 at
 // B = 4096; at D = p = 1024, 11.1 / 14.1 against 15.6 / 18.5 us at B = 1 / 256, even at B = 4096;
 // at D = 2 p = 2048, 9.2 / 12.5 / 70.3 against 13.0 / 18.8 / 121.8 us at B = 1 / 256 / 4096, and
 // at D = 2 p = 8192, 13.4 / 25.8 / 229.5 against 18.1 / 33.5 / 321.1)
 bool circ_bwd_fused_supported(int p, int D, int64_t B) {
-  return (p == 512 && D == 4096) || (p == 1024 && D == 4096) || (p == 128 && D == 4096 && B >= 64) ||
+  (void)B;
+  return (p == 512 && D == 4096) || (p == 1024 && D == 4096) || (p == 128 && D == 4096) ||
          ((D == p || D == 2 * p) && p >= 512);
 }
 

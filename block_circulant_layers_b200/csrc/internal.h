@@ -49,7 +49,7 @@ struct GcSink {
 
 // Backward in one kernel (grad_x and the grad_c cross-spectrum from one transform of g
 // and x per input-block group) for the shapes it covers (circ_bwd_fused_supported: D = 4096
-// at p = 512 or 1024, at p = 128 from B = 64, and layers of one or two blocks, D in {p, 2p},
+// at p = 128, 512 or 1024, and layers of one or two blocks, D in {p, 2p},
 // p >= 512); the caller runs the in-place rdIFFT of grad_c after it.
 bool circ_bwd_fused_supported(int p, int D, int64_t B);
 // Reads and clears the error word of the fused backward (bit 0: a bounded wait for its staged

@@ -38,6 +38,15 @@ inline int layer_x_tokens(int64_t B, int q, int qi_max, int n_sm, int tt_max) {
   return 1;
 }
 
+// Token tiles of the one-kernel backward (circ_bwd_fused.cu): the smaller of its two tile
+// sizes (tt_small tokens) while every CTA of the njgroups block groups then holds one tile
+// and they all fit in one wave (the kernel runs one CTA per SM); the larger one above. With
+// few tokens a CTA's time is one tile's latency, and a smaller tile has less of it (D=4096,
+// p=512: 17.4 against 23.1 us at B = 128; p=1024: 14.6 against 16.8 us at B = 128).
+inline bool layer_fused_small_tiles(int64_t B, int tt_small, int njgroups, int n_sm) {
+  return ((B + tt_small - 1) / tt_small) * njgroups <= n_sm;
+}
+
 // Input blocks per grad_c CTA group: a divisor of q, at most 8, with at most
 // max_slots complex accumulators per CTA (hb bins x q output blocks x QJ), and fewer
 // while ntiles token tiles times q / QJ groups would cover fewer than half the SMs

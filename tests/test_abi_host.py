@@ -159,7 +159,7 @@ def test_deterministic_backward_workspace_size(lib):
     assert workspace_size(lib, 4, 4096, 128, dtype=3) == (EDTYPE, 0)
     assert workspace_size(lib, 0, 4096, 128) == (OK, 0)              # empty batch
     assert workspace_size(lib, 1, 4096, 128) == (OK, 0)              # one slice stores grad_c
-    assert workspace_size(lib, 3, 4096, 512) == (OK, 0)
+    assert workspace_size(lib, 2, 4096, 512) == (OK, 0)              # one tile of 2 tokens
     # D = 4096, p = 128, B = 256: 4 input-block groups x 32 slices of two 4-token tiles, both
     # with grad_x (one kernel) and without (the grad_c kernel); 32 x 512 KiB
     assert workspace_size(lib, 256, 4096, 128) == (OK, 32 * 32 * 32 * 128 * 4)

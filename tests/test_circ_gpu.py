@@ -92,21 +92,23 @@ def test_config_d4096_p128(rd, B, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("B", [1, 3, 5, 9, 37])
+@pytest.mark.parametrize("B", [1, 3, 5, 9, 37, 149, 297, 301])
 @pytest.mark.parametrize("p", [512, 1024])
 def test_fused_backward_shapes(rd, p, B, dtype):
     """D = 4096 at p = 512 (q = 8) and p = 1024 (q = 4): circ_bwd computes grad_x and grad_c
     in one kernel (the cross-spectrum accumulated in tensor memory). Ragged token counts:
-    one CTA storing grad_c, and several adding into it."""
+    one CTA storing grad_c, and several adding into it; the smaller token tiles (2 tokens at
+    p = 512 up to 296 tokens, 1 at p = 1024 up to 148) and the larger ones beyond."""
     check_all(rd, B, 4096, p, dtype, (110 + p, 120 + B, 130 + B))
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
-@pytest.mark.parametrize("B", [64, 77, 256, 259, 301])
+@pytest.mark.parametrize("B", [1, 3, 8, 16, 33, 64, 77, 256, 259, 301])
 def test_fused_backward_p128_block_groups(rd, B, dtype):
-    """D = 4096 at p = 128 (q = 32) from 64 tokens: the fused backward splits the input
+    """D = 4096 at p = 128 (q = 32) at any batch size: the fused backward splits the input
     blocks into 4 groups (grid y), each CTA transforming g in full and x for its group, with
-    a ragged last token tile and several token slices adding into grad_c."""
+    a ragged last token tile and several token slices adding into grad_c; tiles of 2 tokens
+    up to 74 tokens (one tile per CTA in one wave), of 4 above."""
     check_all(rd, B, 4096, 128, dtype, (150, 151 + B, 152 + B))
 
 
@@ -128,11 +130,10 @@ def test_fused_backward_two_blocks(rd, p, B, dtype):
     check_all(rd, B, 2 * p, p, dtype, (190 + p // 512, 191 + B, 192 + B))
 
 
-@pytest.mark.parametrize("p", [512, 4096])
-def test_fused_backward_one_block_stores_every_grad_c_element(rd, p):
-    """q = 1 with one CTA (a few tokens): grad_c is stored, not added; a NaN-filled grad_c
-    must come out finite and right."""
-    B = 3
+@pytest.mark.parametrize("p,B", [(512, 3), (4096, 2)])
+def test_fused_backward_one_block_stores_every_grad_c_element(rd, p, B):
+    """q = 1 with one CTA (one token tile: 4 tokens at p = 512, 2 at p = 4096): grad_c is
+    stored, not added; a NaN-filled grad_c must come out finite and right."""
     c, x, g = make_layer(B, p, p, "bf16", (180, 181, 182))
     c_hat = rd.circ_prepare(to_device(c, "f32"))
     gc = torch.full(c_hat.shape, float("nan"), device="cuda")
@@ -144,11 +145,11 @@ def test_fused_backward_one_block_stores_every_grad_c_element(rd, p):
     assert_parity(to_host_f64(gx), gx_ref, "bf16", "one-block grad_x")
 
 
-@pytest.mark.parametrize("p", [512, 1024])
-def test_fused_backward_stores_every_grad_c_element(rd, p):
-    """With a single CTA (few tokens) the fused kernel stores grad_c instead of adding into a
-    zeroed buffer: a grad_c full of NaN must come out finite and right."""
-    B, D = 3, 4096
+@pytest.mark.parametrize("p,B", [(512, 1), (512, 2), (1024, 1)])
+def test_fused_backward_stores_every_grad_c_element(rd, p, B):
+    """With a single CTA (one token tile) the fused kernel stores grad_c instead of adding
+    into a zeroed buffer: a grad_c full of NaN must come out finite and right."""
+    D = 4096
     c, x, g = make_layer(B, D, p, "bf16", (140, 141, 142))
     c_hat = rd.circ_prepare(to_device(c, "f32"))
     gc = torch.full(c_hat.shape, float("nan"), device="cuda")

@@ -132,3 +132,13 @@ def test_forward_token_tiles(emu):
                     for t2 in (2 * tt, 4 * tt):
                         if t2 <= tt_max:
                             assert emu.rdfft_layer_qi(q, 8, -(-B // t2), N_SM) != full
+
+
+def test_fused_backward_token_tiles(emu):
+    """The one-kernel backward takes its smaller token tile while every CTA then holds one
+    tile and all fit in one wave of one CTA per SM."""
+    f = emu.rdfft_layer_fused_small_tiles
+    f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    assert f(256, 2, 1, N_SM) == 1 and f(296, 2, 1, N_SM) == 1 and f(297, 2, 1, N_SM) == 0   # p = 512
+    assert f(148, 1, 1, N_SM) == 1 and f(149, 1, 1, N_SM) == 0                             # p = 1024
+    assert f(74, 2, 4, N_SM) == 1 and f(75, 2, 4, N_SM) == 0 and f(256, 2, 4, N_SM) == 0   # p = 128
