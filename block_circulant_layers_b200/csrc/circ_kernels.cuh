@@ -785,11 +785,10 @@ static cudaError_t run_gc(const void* g, const void* x, float* grad_c, int64_t B
 // grad_c launcher: a CTA of 512 threads keeps S for QJ input blocks in registers,
 // RI x RJ (output, input) blocks of one bin per thread-slot, NG slots per thread,
 // at most 32 complex accumulators per thread.
-template <int P, typename T>
-static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int64_t B, int q,
-                               cudaStream_t s, GcSink* sink) {
+template <int P, typename T, int TT>
+static cudaError_t launch_gc_tt(const void* g, const void* x, float* grad_c, int64_t B, int q,
+                                cudaStream_t s, GcSink* sink) {
   constexpr int NT = 512;
-  constexpr int TT = (P >= 2048) ? 1 : (P >= 1024 ? 2 : 4);
   constexpr int HB = P / 2;
   const int QJ = layer_qj(q, HB, 32LL * NT, (B + TT - 1) / TT, num_sms());
   if ((int64_t)HB * q * QJ > 32LL * NT) return cudaErrorInvalidConfiguration;
@@ -810,6 +809,20 @@ static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int6
   if (slots <= 8LL * NT) return run_gc<P, T, NT, TT, 8, 1, 1>(g, x, grad_c, B, q, QJ, s, sink);
   if (slots <= 16LL * NT) return run_gc<P, T, NT, TT, 16, 1, 1>(g, x, grad_c, B, q, QJ, s, sink);
   return run_gc<P, T, NT, TT, 32, 1, 1>(g, x, grad_c, B, q, QJ, s, sink);
+}
+
+// Token tiles of 4 (p <= 512), 2 (p = 1024) or 1 token, or half of that while a handful of
+// tokens leaves the SMs idle (layer_gc_half_tiles: grad_c alone at D=4096, B=16: 11.3 against
+// 14.2 us at p = 128, 10.3 against 12.3 at p = 512, 10.2 against 11.4 at p = 1024).
+template <int P, typename T>
+static cudaError_t launch_gc_p(const void* g, const void* x, float* grad_c, int64_t B, int q,
+                               cudaStream_t s, GcSink* sink) {
+  constexpr int TT = (P >= 2048) ? 1 : (P >= 1024 ? 2 : 4);
+  if constexpr (TT > 1) {
+    if (layer_gc_half_tiles(B, TT, q, P / 2, 32LL * 512, num_sms()))
+      return launch_gc_tt<P, T, TT / 2>(g, x, grad_c, B, q, s, sink);
+  }
+  return launch_gc_tt<P, T, TT>(g, x, grad_c, B, q, s, sink);
 }
 
 // Per-p entry of the layer, instantiated once per translation unit (circ_p*.cu):

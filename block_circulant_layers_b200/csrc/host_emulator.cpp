@@ -315,6 +315,9 @@ int rdfft_layer_x_tokens(int64_t B, int q, int qi_max, int n_sm, int tt_max) {
 int rdfft_layer_fused_small_tiles(int64_t B, int tt_small, int njgroups, int n_sm) {
   return rdfft::layer_fused_small_tiles(B, tt_small, njgroups, n_sm) ? 1 : 0;
 }
+int rdfft_layer_gc_half_tiles(int64_t B, int tt, int q, int hb, int64_t max_slots, int n_sm) {
+  return rdfft::layer_gc_half_tiles(B, tt, q, hb, max_slots, n_sm) ? 1 : 0;
+}
 int rdfft_layer_gc_slices(int njgroups, int64_t ntiles, int n_sm, int64_t* tiles_per) {
   return rdfft::layer_gc_slices(njgroups, ntiles, n_sm, tiles_per);
 }

@@ -58,6 +58,19 @@ inline int layer_qj(int q, int hb, int64_t max_slots, int64_t ntiles, int n_sm) 
   return qj;
 }
 
+// Token tiles of the grad_c kernel: half of tt while the half-size tiles number at most half
+// the SMs and their grid (tiles times the input-block groups layer_qj then sets) fits one
+// wave; with that few tokens each CTA's time is one tile's latency, and a smaller tile has
+// less of it. Above, the full tiles (more tokens per c_hat-free pass over g and x).
+inline bool layer_gc_half_tiles(int64_t B, int tt, int q, int hb, int64_t max_slots, int n_sm) {
+  const int th = tt / 2;
+  if (th < 1) return false;
+  const int64_t nt = (B + th - 1) / th;
+  if (nt > n_sm / 2) return false;
+  const int qj = layer_qj(q, hb, max_slots, nt, n_sm);
+  return nt * (q / qj) <= n_sm;
+}
+
 // Token slices of the persistent grad_c grid: about n_sm CTAs over the njgroups
 // input-block groups, each slice a whole number of token tiles (*tiles_per, at least
 // 1). Returns the number of slices (at least 1).

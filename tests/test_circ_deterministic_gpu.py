@@ -79,7 +79,7 @@ def test_deterministic_grad_c(rd, B, D, p, with_gx, dtype):
     assert_parity(to_host_f64(gc2), gc_ref, dtype, f"circ_bwd grad_c B={B} D={D} p={p}")
 
 
-@pytest.mark.parametrize("B,D,p", [(1, 4096, 128), (2, 4096, 512), (1, 4096, 1024), (2, 1024, 1024), (3, 512, 64)])
+@pytest.mark.parametrize("B,D,p", [(1, 4096, 128), (2, 4096, 512), (1, 4096, 1024), (2, 1024, 1024), (2, 512, 64)])
 def test_one_slice_needs_no_workspace(rd, B, D, p):
     """A handful of tokens: one slice per block group stores grad_c, no workspace, and the
     result equals circ_bwd's bit for bit."""

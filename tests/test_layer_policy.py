@@ -142,3 +142,25 @@ def test_fused_backward_token_tiles(emu):
     assert f(256, 2, 1, N_SM) == 1 and f(296, 2, 1, N_SM) == 1 and f(297, 2, 1, N_SM) == 0   # p = 512
     assert f(148, 1, 1, N_SM) == 1 and f(149, 1, 1, N_SM) == 0                             # p = 1024
     assert f(74, 2, 4, N_SM) == 1 and f(75, 2, 4, N_SM) == 0 and f(256, 2, 4, N_SM) == 0   # p = 128
+
+
+def test_grad_c_token_tiles(emu):
+    """The grad_c kernel halves its token tile while that leaves at most half the SMs' worth of
+    tiles and its grid fits one wave."""
+    f = emu.rdfft_layer_gc_half_tiles
+    f.argtypes = [ctypes.c_int64, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_int]
+    S = 32 * 512
+    # D = 4096: p = 512 (q = 8, 256 bins), p = 128 (q = 32, 64 bins), p = 1024 (q = 4, 512 bins)
+    assert f(16, 4, 8, 256, S, N_SM) == 1 and f(128, 4, 8, 256, S, N_SM) == 1
+    assert f(256, 4, 8, 256, S, N_SM) == 0
+    assert f(16, 4, 32, 64, S, N_SM) == 1 and f(64, 4, 32, 64, S, N_SM) == 1
+    assert f(128, 4, 32, 64, S, N_SM) == 0
+    assert f(64, 2, 4, 512, S, N_SM) == 1 and f(128, 2, 4, 512, S, N_SM) == 0
+    assert f(5, 1, 4, 512, S, N_SM) == 0                  # no tile smaller than one token
+    for q, hb in ((1, 2048), (4, 512), (8, 256), (16, 128), (32, 64), (64, 32), (128, 32)):
+        for B in (1, 2, 7, 16, 64, 100, 128, 256, 1000):
+            for tt in (2, 4):
+                if f(B, tt, q, hb, S, N_SM):
+                    nt = -(-B // (tt // 2))
+                    qj = emu.rdfft_layer_qj(q, hb, S, nt, N_SM)
+                    assert nt <= N_SM // 2 and nt * (q // qj) <= N_SM
