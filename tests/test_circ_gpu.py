@@ -286,3 +286,27 @@ def test_grad_c_single_token_slice_writes_every_element(rd, B, D, p):
     assert_parity(to_host_f64(gc), gc_ref, "bf16", f"grad_c B={B} D={D} p={p}")
     assert_parity(to_host_f64(gx), gx_ref, "bf16", f"grad_x B={B} D={D} p={p}")
     assert_parity(to_host_f64(y), oracle.circ_forward(x.exact, c.exact), "bf16", f"y B={B} D={D} p={p}")
+
+
+@pytest.mark.parametrize("D,p,B", [(4096, 512, 31), (4096, 512, 64), (4096, 512, 255), (4096, 512, 256),
+                                   (4096, 512, 512), (2048, 512, 128), (1024, 256, 256), (4096, 256, 64),
+                                   (1024, 64, 64)])
+def test_forward_token_tile_choices(rd, D, p, B):
+    """The forward's token tile (4, 2 or 1 tokens per CTA, the largest whose grid keeps a
+    token's output blocks in one CTA) on both sides of each choice, and the backward beside it."""
+    check_all(rd, B, D, p, "bf16", (500 + p, 501 + B, 502 + D))
+
+
+@pytest.mark.parametrize("D,p,B", [(4096, 128, 16), (4096, 128, 64), (4096, 128, 129), (4096, 512, 16),
+                                   (4096, 512, 148), (4096, 512, 300), (4096, 1024, 64), (4096, 1024, 149),
+                                   (1024, 64, 100), (4096, 256, 77)])
+def test_grad_c_token_tile_choices(rd, D, p, B):
+    """grad_c alone (the grad_c kernel) with half-size token tiles at few tokens and full ones
+    above, against the oracle; a NaN-filled grad_c must come out finite and right."""
+    c, x, g = make_layer(B, D, p, "bf16", (510 + p, 511 + B, 512 + D))
+    c_hat = rd.circ_prepare(to_device(c, "f32"))
+    gc = torch.full(c_hat.shape, float("nan"), device="cuda")
+    rd.circ_bwd(to_device(g, "bf16"), to_device(x, "bf16"), c_hat, p, grad_c=gc, need_grad_x=False)
+    torch.cuda.synchronize()
+    _, gc_ref = oracle.circ_backward(g.exact, x.exact, c.exact)
+    assert_parity(to_host_f64(gc), gc_ref, "bf16", f"grad_c alone B={B} D={D} p={p}")
