@@ -155,3 +155,45 @@ def test_layer_chain_without_sync(rd):
     assert torch.equal(gx0.view(torch.int16), gx1.view(torch.int16))
     # grad_c is a sum over token slices added with atomics: order may differ
     assert np.allclose(gc0.cpu().numpy(), gc1.cpu().numpy(), rtol=1e-5, atol=1e-6 * gc0.abs().max().item())
+
+
+def _chain_layer_det(rd, bufs, p):
+    """prepare -> forward -> deterministic backward -> rdFFT of grad_c's rows, twice: the
+    second backward overwrites grad_c and the workspace while the grid before it may still be
+    draining (programmatic dependent launch)."""
+    c, x, g, ch, y, gx, gc, ws, spec = bufs
+    ops = []
+    for _ in range(2):
+        ops.append(lambda: rd.circ_prepare(c, out=ch))
+        ops.append(lambda: rd.circ_fwd(x, ch, p, y=y))
+        ops.append(lambda: rd.circ_bwd(g, x, ch, p, grad_x=gx, grad_c=gc, deterministic=True, workspace=ws))
+        ops.append(lambda: spec.copy_(gc))
+        ops.append(lambda: rd.rdfft_fwd(spec, p))
+    return ops
+
+
+@pytest.mark.parametrize("mode", ["stream", "graph"])
+@pytest.mark.parametrize("D,p,B", [(4096, 128, 256), (4096, 512, 64), (1024, 1024, 256), (1024, 64, 300)])
+def test_deterministic_layer_chain_without_sync(rd, D, p, B, mode):
+    """The deterministic backward chained with the layer's other calls, in a stream and in a
+    captured CUDA graph, gives the same bits as the synchronised sequence: the zeroing,
+    per-slice, ordered-sum and rdIFFT launches keep their order without a host sync."""
+    q = D // p
+
+    def make():
+        c = torch.from_numpy(sample(83_000 + p, (q, q, p), "f32", sigma=D ** -0.5).stored).cuda()
+        x = to_device(sample(83_001 + B, (B, D), "bf16"), "bf16")
+        g = to_device(sample(83_002 + B, (B, D), "bf16"), "bf16")
+        need = max(16, rd.circ_bwd_workspace_size(B, D, p, torch.bfloat16))
+        ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+        return [c, x, g, torch.empty_like(c), torch.empty_like(x), torch.empty_like(x), torch.empty_like(c), ws,
+                torch.empty_like(c)]
+
+    ref = make()
+    _run_synced(_chain_layer_det(rd, ref, p))
+    got = make()
+    _run_chained(_chain_layer_det(rd, got, p), mode, _chain_layer_det(rd, make(), p))
+    for name, i in (("y", 4), ("grad_x", 5)):
+        assert torch.equal(got[i].view(torch.int16), ref[i].view(torch.int16)), f"{name} ({D}, {p}, {B}, {mode})"
+    for name, i in (("grad_c", 6), ("rdFFT of grad_c", 8)):
+        assert torch.equal(got[i], ref[i]), f"{name} ({D}, {p}, {B}, {mode})"
